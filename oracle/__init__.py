@@ -1,0 +1,7 @@
+"""fp64 CPU oracle for the Sol-Attn forward operator: test infrastructure only.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package. It shares no code with the CUDA path.
+"""
+from .solattn_ref import (MODES, forward, keep_sets, kept_per_head, pool, proxy,  # noqa: F401
+                          sample_qblocks, valid_counts, visit_order)

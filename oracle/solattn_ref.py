@@ -1,0 +1,258 @@
+"""Plain fp64 CPU oracle for the Sol-Attn forward operator.
+
+TEST INFRASTRUCTURE ONLY. Nothing in the product path imports this module:
+only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may call it. It shares no code with the CUDA path.
+
+What it computes (one query block i of one (batch, head) pair; rows R_i,
+n_i = |R_i|; key blocks j with columns C_j, n_j = |C_j|; d = head dim):
+
+1. Pool: q_i = mean of Q over R_i, k_j and v_j = means of K and V over C_j,
+   over the valid rows only ("the proxy score for each query-key block pair is
+   derived from the means of the corresponding query and key blocks":
+   paperlayer summary "Sol-Attn: Accelerating Video Generation Inference via
+   On-the-Fly Attention Sparsification", §2 Preliminaries, Block-Sparse
+   Attention).
+2. Proxy: s_ij = q_i . k_j / sqrt(d).
+3. Visit order: key blocks are visited starting at the block holding query
+   block i's first token, ascending with wrap-around. The pages do not state an
+   order; this is the reading adopted for this build (local attention in video
+   DiTs puts the largest proxies near the diagonal).
+4. Threshold (on-the-fly block thresholding, paperlayer summary §3
+   Methodology, "On-the-fly sparsification"; abstract "comparing block proxy
+   scores against a threshold during online softmax"): M(t) is the running
+   maximum of the proxies visited so far including the current one, and the
+   visited block is kept iff s >= M(t) - tau. The pages' own threshold is a
+   query-dependent mean + beta * std; the running-max form is the reading
+   fixed for this build.
+5. Output, closed form (no online recurrence):
+   keep_correct: O_r = [sum_{j kept} sum_{c in C_j} e^{s_rc} v_c
+                        + sum_{j dropped} n_j e^{s_ij} v_j]
+                       / [sum_{j kept} sum_{c in C_j} e^{s_rc}
+                        + sum_{j dropped} n_j e^{s_ij}]
+   (zeroth-order proxy-score reuse with pooled keys and summed values:
+   paperlayer summary §3 Methodology, "Approximate correction", and App. B,
+   "Approximation error"); keep_drop drops the dropped-block terms (abstract,
+   "keep-or-drop sparsification"); dense keeps every block.
+6. Stats: kept blocks per (b, h) = sum over query blocks of |K_i|.
+
+All arithmetic is float64 on the exact bf16 input values.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+MODES = {"dense": 0, "keep_drop": 1, "keep_correct": 2}
+MODE_NAMES = {v: k for k, v in MODES.items()}
+
+
+def _mode_name(mode):
+    if isinstance(mode, str):
+        if mode not in MODES:
+            raise ValueError(f"unknown mode {mode!r}")
+        return mode
+    return MODE_NAMES[int(mode)]
+
+
+def as_f64(x) -> np.ndarray:
+    """A torch tensor (any dtype, any device) or array -> float64 numpy array."""
+    if hasattr(x, "detach"):
+        x = x.detach().to("cpu")
+        import torch
+        x = x.to(torch.float64).numpy()
+    return np.asarray(x, dtype=np.float64)
+
+
+# ----------------------------------------------------------------- step 1
+
+def n_blocks(N: int, blk: int) -> int:
+    return -(-N // blk)
+
+
+def block_rows(N: int, blk: int, j: int) -> slice:
+    """Rows of block j: [j*blk, min(N, (j+1)*blk))."""
+    return slice(j * blk, min(N, (j + 1) * blk))
+
+
+def valid_counts(N: int, blk: int) -> np.ndarray:
+    """n_j: number of valid rows of each block (the last one may be ragged)."""
+    return np.array([block_rows(N, blk, j).stop - j * blk for j in range(n_blocks(N, blk))],
+                    dtype=np.int64)
+
+
+def pool(x: np.ndarray, blk: int) -> np.ndarray:
+    """Block means over the valid rows: [..., N, d] -> [..., nB, d] (float64)."""
+    x = as_f64(x)
+    N = x.shape[-2]
+    out = np.empty(x.shape[:-2] + (n_blocks(N, blk), x.shape[-1]), dtype=np.float64)
+    for j in range(n_blocks(N, blk)):
+        rows = x[..., block_rows(N, blk, j), :]
+        out[..., j, :] = rows.sum(axis=-2) / rows.shape[-2]
+    return out
+
+
+# ----------------------------------------------------------------- step 2
+
+def proxy(qbar: np.ndarray, kbar: np.ndarray) -> np.ndarray:
+    """s_ij = q_i . k_j / sqrt(d): [..., nQB, d] x [..., nKB, d] -> [..., nQB, nKB]."""
+    d = qbar.shape[-1]
+    return np.matmul(qbar, np.swapaxes(kbar, -1, -2)) / math.sqrt(d)
+
+
+# ----------------------------------------------------------------- step 3
+
+def diagonal_block(i: int, Bq: int, Bk: int, nKB: int) -> int:
+    """The key block holding query block i's first token (clamped to the last block)."""
+    return min((i * Bq) // Bk, nKB - 1)
+
+
+def visit_order(i: int, nKB: int, Bq: int, Bk: int, order: str = "rotated") -> np.ndarray:
+    """pi_i(t), t = 0..nKB-1: the key blocks in the order query block i visits them."""
+    if order == "natural":
+        return np.arange(nKB, dtype=np.int64)
+    if order != "rotated":
+        raise ValueError(order)
+    j0 = diagonal_block(i, Bq, Bk, nKB)
+    return (j0 + np.arange(nKB, dtype=np.int64)) % nKB
+
+
+# ----------------------------------------------------------------- step 4
+
+def keep_test(s_visited: np.ndarray, running_max: np.ndarray, tau: float) -> np.ndarray:
+    """Keep iff the proxy clears the running maximum minus tau."""
+    return s_visited >= running_max - tau
+
+
+def route_row(s_row: np.ndarray, visit: np.ndarray, tau: float):
+    """Keep flags and threshold margins of one query block.
+
+    s_row: [nKB] proxies of query block i; visit: the visit order.
+    Returns (keep [nKB] bool, margin [nKB] = s - (M(t) - tau) at visit time).
+    """
+    s_vis = s_row[visit]
+    running_max = np.maximum.accumulate(s_vis)
+    keep_vis = keep_test(s_vis, running_max, tau)
+    keep = np.zeros(s_row.shape[0], dtype=bool)
+    keep[visit] = keep_vis
+    margin = np.empty(s_row.shape[0], dtype=np.float64)
+    margin[visit] = s_vis - (running_max - tau)
+    return keep, margin
+
+
+def keep_sets(q, k, Bq: int, Bk: int, tau: float, mode="keep_correct", order: str = "rotated"):
+    """Keep sets of every query block.
+
+    Returns (keep [B, H, nQB, nKB] bool, margin [B, H, nQB, nKB] float64,
+    sbar [B, H, nQB, nKB] float64). In dense mode every block is kept and the
+    margin is +inf.
+    """
+    mode = _mode_name(mode)
+    q = as_f64(q)
+    k = as_f64(k)
+    B, H, N, d = q.shape
+    nQB, nKB = n_blocks(N, Bq), n_blocks(N, Bk)
+    sbar = proxy(pool(q, Bq), pool(k, Bk))
+    keep = np.ones((B, H, nQB, nKB), dtype=bool)
+    margin = np.full((B, H, nQB, nKB), np.inf)
+    if mode == "dense" or tau == math.inf:
+        return keep, margin, sbar
+    for i in range(nQB):
+        visit = visit_order(i, nKB, Bq, Bk, order)
+        for b in range(B):
+            for h in range(H):
+                keep[b, h, i], margin[b, h, i] = route_row(sbar[b, h, i], visit, tau)
+    return keep, margin, sbar
+
+
+def kept_per_head(keep: np.ndarray) -> np.ndarray:
+    """Sum of |K_i| over the query blocks of each (b, h): int64 [B, H]."""
+    return keep.sum(axis=(-1, -2)).astype(np.int64)
+
+
+# ----------------------------------------------------------------- step 5
+
+def correction_terms(sbar_row: np.ndarray, dropped: np.ndarray, counts: np.ndarray,
+                     vbar: np.ndarray):
+    """Pseudo-key logits, weights and values of the dropped blocks of one query block.
+
+    Each dropped block j enters as one pseudo-key with logit s_ij, multiplicity
+    n_j and value v_j (its mean V): weight n_j * e^{s_ij}.
+    Returns (logits [m], multiplicities [m], values [m, d]).
+    """
+    idx = np.nonzero(dropped)[0]
+    return sbar_row[idx], counts[idx].astype(np.float64), vbar[idx]
+
+
+def attend_block(q_rows, k, v, kept_cols, pseudo):
+    """Closed-form weighted softmax of one query block.
+
+    q_rows [n_i, d]; k, v [N, d]; kept_cols: bool [N]; pseudo = (logits,
+    multiplicities, values) of the pseudo-keys or None.
+    """
+    d = q_rows.shape[-1]
+    s = (q_rows @ k[kept_cols].T) / math.sqrt(d)          # [n_i, n_kept]
+    m = s.max(axis=1) if s.shape[1] else np.full(q_rows.shape[0], -np.inf)
+    if pseudo is not None and pseudo[0].size:
+        m = np.maximum(m, pseudo[0].max())
+    e = np.exp(s - m[:, None])
+    num = e @ v[kept_cols]
+    den = e.sum(axis=1)
+    if pseudo is not None and pseudo[0].size:
+        logits, mult, vals = pseudo
+        w = mult[None, :] * np.exp(logits[None, :] - m[:, None])   # [n_i, m]
+        num = num + w @ vals
+        den = den + w.sum(axis=1)
+    return num / den[:, None]
+
+
+def forward(q, k, v, Bq: int, Bk: int, tau: float, mode="keep_correct", order: str = "rotated",
+            keep: np.ndarray | None = None, qblocks=None):
+    """Sol-Attn output in float64.
+
+    q, k, v: [B, H, N, d] (bf16 torch tensors or arrays; converted exactly).
+    keep: optional [B, H, nQB, nKB] override of the keep sets (used to compare
+    outputs on the GPU's own keep set where a near-threshold proxy flipped).
+    qblocks: None for every query block, or an iterable of (b, h, i) triples.
+    Returns (out [B, H, N, d] float64 with NaN rows for query blocks that were
+    not computed, keep [B, H, nQB, nKB]).
+    """
+    mode = _mode_name(mode)
+    q, k, v = as_f64(q), as_f64(k), as_f64(v)
+    B, H, N, d = q.shape
+    nQB, nKB = n_blocks(N, Bq), n_blocks(N, Bk)
+    if keep is None:
+        keep, _, sbar = keep_sets(q, k, Bq, Bk, tau, mode, order)
+    else:
+        keep = np.asarray(keep, dtype=bool)
+        sbar = proxy(pool(q, Bq), pool(k, Bk))
+    if mode == "dense":
+        keep = np.ones_like(keep)
+    counts = valid_counts(N, Bk)
+    vbar = pool(v, Bk) if mode == "keep_correct" else None
+    col_block = np.arange(N) // Bk
+    out = np.full(q.shape, np.nan)
+    if qblocks is None:
+        qblocks = [(b, h, i) for b in range(B) for h in range(H) for i in range(nQB)]
+    for b, h, i in qblocks:
+        rows = block_rows(N, Bq, i)
+        kept_cols = keep[b, h, i][col_block]
+        pseudo = None
+        if mode == "keep_correct":
+            pseudo = correction_terms(sbar[b, h, i], ~keep[b, h, i], counts, vbar[b, h])
+        out[b, h, rows] = attend_block(q[b, h, rows], k[b, h], v[b, h], kept_cols, pseudo)
+    return out, keep
+
+
+def sample_qblocks(B, H, nQB, Bq, Bk, nKB, per_head=64, seed=0):
+    """Seeded sample of query blocks per head, plus block 0, the last (ragged) one and
+    the blocks whose diagonal is at the extremes."""
+    rng = np.random.default_rng(seed)
+    picks = []
+    for b in range(B):
+        for h in range(H):
+            chosen = set(int(x) for x in rng.choice(nQB, size=min(per_head, nQB), replace=False))
+            chosen.update({0, nQB - 1, nQB // 2})
+            picks.extend((b, h, i) for i in sorted(chosen))
+    return picks

@@ -1,0 +1,340 @@
+"""Pins of the fp64 oracle to things other than itself.
+
+Each pin checks the oracle against a closed form, a library routine, a
+hand-worked case or a brute-force loop, so that a plausible mistake anywhere in
+the oracle (a dropped term, a wrong scale, sign, index or order) fails at least
+one of them. ``test_planted_mistakes_are_caught`` plants such mistakes in the
+oracle (on the CPU) and checks that the pins catch every one.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle.solattn_ref as ref
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "handworked_d4.json")
+
+
+def _rand(B, H, N, d, seed, scale=1.0):
+    """Q/K with a component shared by runs of 16 tokens (so block means spread and some
+    blocks fall below the threshold) plus per-token noise; V standard normal."""
+    rng = np.random.default_rng(seed)
+
+    def qk():
+        runs = rng.standard_normal((B, H, -(-N // 16), d)) * scale
+        return np.repeat(runs, 16, axis=2)[:, :, :N] + 0.5 * rng.standard_normal((B, H, N, d))
+
+    q, k = qk(), qk()
+    v = rng.standard_normal((B, H, N, d))
+    return q, k, v
+
+
+def _sdpa(q, k, v, mask=None):
+    t = lambda x: torch.from_numpy(np.ascontiguousarray(x))
+    out = torch.nn.functional.scaled_dot_product_attention(
+        t(q), t(k), t(v), attn_mask=None if mask is None else t(mask))
+    return out.numpy()
+
+
+def _token_mask(keep, N, Bq, Bk):
+    """[.., N, N] bool: query token r may see key token c iff its blocks are kept."""
+    rb = np.arange(N) // Bq
+    cb = np.arange(N) // Bk
+    return keep[..., rb, :][..., :, cb]
+
+
+# ------------------------------------------------------------------ pins
+
+def pin_handworked():
+    g = json.load(open(GOLDEN))
+    env = {"ln4": math.log(4.0), "ln2": math.log(2.0), "sqrt2": math.sqrt(2.0)}
+    ev = lambda x: float(eval(str(x), {"__builtins__": {}}, env))  # closed forms only
+    q = np.array([[ev(x) for x in r] for r in g["q"]])[None, None]
+    k = np.array([[ev(x) for x in r] for r in g["k"]])[None, None]
+    v = np.array([[ev(x) for x in r] for r in g["v"]])[None, None]
+    for case in g["cases"]:
+        out, keep = ref.forward(q, k, v, g["Bq"], g["Bk"], case["tau"], case["mode"],
+                                order=case["order"])
+        if case["mode"] != "dense":
+            assert np.array_equal(keep[0, 0].astype(int), np.array(case["keep"])), case
+        for row, vals in case["rows"].items():
+            np.testing.assert_allclose(out[0, 0, int(row)], [ev(x) for x in vals],
+                                       rtol=1e-13, atol=1e-13, err_msg=str(case))
+
+
+def pin_pool_is_block_mean():
+    x = np.random.default_rng(1).standard_normal((2, 3, 203, 8))
+    for blk in (16, 64):
+        p = ref.pool(x, blk)
+        assert p.shape == (2, 3, -(-203 // blk), 8)
+        for j in range(p.shape[2]):
+            np.testing.assert_allclose(p[:, :, j], np.mean(x[:, :, j * blk:(j + 1) * blk], axis=2),
+                                       rtol=1e-14, atol=1e-14)
+
+
+def pin_dense_is_softmax_attention():
+    q, k, v = _rand(1, 2, 200, 16, seed=2, scale=1.5)
+    want = _sdpa(q, k, v)
+    for mode, tau in (("dense", 0.5), ("keep_drop", math.inf), ("keep_correct", math.inf)):
+        out, _ = ref.forward(q, k, v, 32, 48, tau, mode)
+        np.testing.assert_allclose(out, want, rtol=1e-12, atol=1e-12, err_msg=mode)
+
+
+def pin_keep_drop_is_masked_attention():
+    q, k, v = _rand(1, 2, 190, 16, seed=3, scale=1.5)
+    for Bq, Bk, tau in ((32, 32, 1.0), (32, 64, 2.0), (64, 32, 0.5)):
+        out, keep = ref.forward(q, k, v, Bq, Bk, tau, "keep_drop")
+        assert not keep.all()
+        mask = _token_mask(keep, 190, Bq, Bk)
+        np.testing.assert_allclose(out, _sdpa(q, k, v, mask), rtol=1e-12, atol=1e-12)
+
+
+def pin_keep_correct_is_augmented_attention():
+    """keep_correct == softmax attention over the kept keys plus one pseudo-key per
+    dropped block (zero key vector, additive bias s_ij + ln n_j, value = block mean of V)."""
+    N, d = 170, 16
+    q, k, v = _rand(1, 1, N, d, seed=4, scale=1.5)
+    for Bq, Bk, tau in ((32, 32, 1.0), (64, 32, 0.3)):
+        out, keep = ref.forward(q, k, v, Bq, Bk, tau, "keep_correct")
+        assert not keep.all()
+        nQB, nKB = keep.shape[-2:]
+        qb = np.mean  # pooled means via numpy directly (library routine)
+        qbar = np.stack([qb(q[0, 0, i * Bq:(i + 1) * Bq], axis=0) for i in range(nQB)])
+        kbar = np.stack([qb(k[0, 0, j * Bk:(j + 1) * Bk], axis=0) for j in range(nKB)])
+        vbar = np.stack([qb(v[0, 0, j * Bk:(j + 1) * Bk], axis=0) for j in range(nKB)])
+        counts = np.array([min(N, (j + 1) * Bk) - j * Bk for j in range(nKB)])
+        sbar = np.einsum("id,jd->ij", qbar, kbar) / math.sqrt(d)
+        keys = np.concatenate([k[0, 0], np.zeros((nKB, d))])
+        vals = np.concatenate([v[0, 0], vbar])
+        bias = np.full((N, N + nKB), -np.inf)
+        rb, cb = np.arange(N) // Bq, np.arange(N) // Bk
+        kp = keep[0, 0]
+        bias[:, :N] = np.where(kp[rb][:, cb], 0.0, -np.inf)
+        bias[:, N:] = np.where(kp[rb], -np.inf, sbar[rb] + np.log(counts)[None, :])
+        want = _sdpa(q[0, 0][None], keys[None], vals[None], bias[None])[0]
+        np.testing.assert_allclose(out[0, 0], want, rtol=1e-12, atol=1e-12)
+
+
+def pin_constant_blocks_correction_exact():
+    """Zero centred score spread (constant Q rows per query block, constant K rows per
+    key block) makes the zeroth-order correction exact: keep_correct == dense for every tau
+    (paperlayer summary, App. B: the error vanishes with the score spread)."""
+    rng = np.random.default_rng(5)
+    N, d = 150, 8
+    for Bq, Bk in ((32, 32), (32, 64), (64, 32)):
+        nQB, nKB = -(-N // Bq), -(-N // Bk)
+        q = np.repeat(rng.standard_normal((nQB, d)) * 2.0, Bq, axis=0)[:N][None, None]
+        k = np.repeat(rng.standard_normal((nKB, d)) * 2.0, Bk, axis=0)[:N][None, None]
+        v = rng.standard_normal((1, 1, N, d))
+        dense, _ = ref.forward(q, k, v, Bq, Bk, 0.0, "dense")
+        for tau in (0.0, 0.5, 2.0, math.inf):
+            out, keep = ref.forward(q, k, v, Bq, Bk, tau, "keep_correct")
+            np.testing.assert_allclose(out, dense, rtol=1e-12, atol=1e-12)
+        assert not ref.keep_sets(q, k, Bq, Bk, 0.5)[0].all()
+
+
+def pin_constant_v_is_reproduced():
+    q, k, _ = _rand(1, 2, 130, 8, seed=6, scale=2.0)
+    v = np.broadcast_to(np.array([1.5, -2.0, 0.25, 3.0, 0.0, 1.0, -1.0, 7.0]), q.shape).copy()
+    for mode in ("dense", "keep_drop", "keep_correct"):
+        out, _ = ref.forward(q, k, v, 32, 32, 0.5, mode)
+        np.testing.assert_allclose(out, v, rtol=1e-13, atol=1e-13)
+
+
+def pin_tau_zero_keeps_records():
+    """tau = 0 keeps exactly the record positions of the visit sequence: position t is
+    kept iff its proxy is >= every earlier proxy (ties included; brute force pairwise)."""
+    rng = np.random.default_rng(7)
+    N, d, Bq, Bk = 320, 8, 32, 32
+    q = rng.standard_normal((1, 1, N, d))
+    palette = rng.integers(-2, 3, size=(3, d)).astype(float)  # 3 distinct pooled keys
+    k = np.repeat(palette[rng.integers(0, 3, size=N // Bk)], Bk, axis=0)[None, None]
+    keep, _, sbar = ref.keep_sets(q, k, Bq, Bk, 0.0)
+    nQB, nKB = keep.shape[-2:]
+    for i in range(nQB):
+        j0 = min(i * Bq // Bk, nKB - 1)
+        seq = [(j0 + t) % nKB for t in range(nKB)]
+        for t, j in enumerate(seq):
+            record = all(sbar[0, 0, i, j] >= sbar[0, 0, i, jp] for jp in seq[:t])
+            assert keep[0, 0, i, j] == record, (i, t)
+    # exact ties occur in this input (repeated pooled keys), and some are kept
+    assert all(len(set(sbar[0, 0, i].tolist())) <= 3 for i in range(nQB))
+    assert keep.sum() > nQB
+
+
+def pin_keep_set_structure():
+    q, k, _ = _rand(2, 2, 260, 16, seed=8, scale=2.0)
+    prev = None
+    for tau in (0.0, 0.5, 1.0, 2.0, 4.0, math.inf):
+        keep, margin, _ = ref.keep_sets(q, k, 32, 64, tau)
+        nQB, nKB = keep.shape[-2:]
+        for i in range(nQB):
+            assert keep[:, :, i, min(i * 32 // 64, nKB - 1)].all()  # first visit kept
+        if prev is not None:
+            assert (keep | ~prev).all()  # monotone: kept at smaller tau => kept
+        if tau == math.inf:
+            assert keep.all()
+        else:
+            assert np.array_equal(keep, margin >= 0)
+        prev = keep
+
+
+def pin_visit_order():
+    for N, Bq, Bk in ((1000, 64, 64), (1000, 128, 64), (1000, 64, 128), (130, 64, 128)):
+        nQB, nKB = -(-N // Bq), -(-N // Bk)
+        for i in range(nQB):
+            vo = ref.visit_order(i, nKB, Bq, Bk)
+            assert sorted(vo.tolist()) == list(range(nKB))
+            first_tok = i * Bq
+            assert vo[0] == min(first_tok // Bk, nKB - 1)  # block holding the first token
+            assert all((vo[t + 1] - vo[t]) % nKB == 1 for t in range(nKB - 1))
+
+
+def _brute_force(q, k, v, Bq, Bk, tau, mode):
+    """Pure-Python scalar loops over one head: the definition written out."""
+    N, d = len(q), len(q[0])
+    nQB, nKB = -(-N // Bq), -(-N // Bk)
+
+    def mean(rows):
+        return [sum(r[c] for r in rows) / len(rows) for c in range(d)]
+
+    qb = [mean(q[i * Bq:(i + 1) * Bq]) for i in range(nQB)]
+    kb = [mean(k[j * Bk:(j + 1) * Bk]) for j in range(nKB)]
+    vb = [mean(v[j * Bk:(j + 1) * Bk]) for j in range(nKB)]
+    out = []
+    for r in range(N):
+        i = r // Bq
+        keep = [True] * nKB
+        if mode != "dense":
+            j0 = min(i * Bq // Bk, nKB - 1)
+            best = -math.inf
+            for t in range(nKB):
+                j = (j0 + t) % nKB
+                s = sum(qb[i][c] * kb[j][c] for c in range(d)) / math.sqrt(d)
+                best = max(best, s)
+                keep[j] = s >= best - tau
+        num = [0.0] * d
+        den = 0.0
+        for j in range(nKB):
+            if keep[j]:
+                for col in range(j * Bk, min(N, (j + 1) * Bk)):
+                    w = math.exp(sum(q[r][c] * k[col][c] for c in range(d)) / math.sqrt(d))
+                    den += w
+                    num = [num[c] + w * v[col][c] for c in range(d)]
+            elif mode == "keep_correct":
+                nj = min(N, (j + 1) * Bk) - j * Bk
+                s = sum(qb[i][c] * kb[j][c] for c in range(d)) / math.sqrt(d)
+                w = nj * math.exp(s)
+                den += w
+                num = [num[c] + w * vb[j][c] for c in range(d)]
+        out.append([x / den for x in num])
+    return out
+
+
+def pin_brute_force_tiny():
+    q, k, v = _rand(1, 1, 75, 4, seed=9, scale=1.2)
+    for Bq, Bk, tau in ((16, 16, 0.4), (16, 32, 0.2), (32, 16, 1.0)):
+        for mode in ("dense", "keep_drop", "keep_correct"):
+            out, _ = ref.forward(q, k, v, Bq, Bk, tau, mode)
+            want = _brute_force(q[0, 0].tolist(), k[0, 0].tolist(), v[0, 0].tolist(),
+                                Bq, Bk, tau, mode)
+            np.testing.assert_allclose(out[0, 0], np.array(want), rtol=1e-11, atol=1e-12,
+                                       err_msg=f"{mode} {Bq} {Bk} {tau}")
+
+
+PINS = [pin_handworked, pin_pool_is_block_mean, pin_dense_is_softmax_attention,
+        pin_keep_drop_is_masked_attention, pin_keep_correct_is_augmented_attention,
+        pin_constant_blocks_correction_exact, pin_constant_v_is_reproduced,
+        pin_tau_zero_keeps_records, pin_keep_set_structure, pin_visit_order,
+        pin_brute_force_tiny]
+
+
+@pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
+def test_pin(pin):
+    pin()
+
+
+# -------------------------------------------------------- planted mistakes
+
+def _mut_pool_by_blk(x, blk):
+    x = ref.as_f64(x)
+    N = x.shape[-2]
+    out = np.empty(x.shape[:-2] + (ref.n_blocks(N, blk), x.shape[-1]))
+    for j in range(out.shape[-2]):
+        out[..., j, :] = x[..., j * blk:(j + 1) * blk, :].sum(axis=-2) / blk
+    return out
+
+
+def _mut_proxy_unscaled(qbar, kbar):
+    return np.matmul(qbar, np.swapaxes(kbar, -1, -2))
+
+
+def _mut_visit_natural(i, nKB, Bq, Bk, order="rotated"):
+    return np.arange(nKB, dtype=np.int64)
+
+
+def _mut_diag_index(i, Bq, Bk, nKB):
+    return min(i, nKB - 1)
+
+
+def _mut_keep_strict(s, m, tau):
+    return s > m - tau
+
+
+def _mut_corr_no_multiplicity(sbar_row, dropped, counts, vbar):
+    idx = np.nonzero(dropped)[0]
+    return sbar_row[idx], np.ones(idx.size), vbar[idx]
+
+
+def _mut_corr_summed_value(sbar_row, dropped, counts, vbar):
+    idx = np.nonzero(dropped)[0]
+    return sbar_row[idx], counts[idx].astype(float), vbar[idx] * counts[idx][:, None]
+
+
+def _mut_attend_no_pseudo_den(q_rows, k, v, kept_cols, pseudo):
+    d = q_rows.shape[-1]
+    s = (q_rows @ k[kept_cols].T) / math.sqrt(d)
+    m = s.max(axis=1)
+    e = np.exp(s - m[:, None])
+    num, den = e @ v[kept_cols], e.sum(axis=1)
+    if pseudo is not None and pseudo[0].size:
+        logits, mult, vals = pseudo
+        w = mult[None, :] * np.exp(logits[None, :] - m[:, None])
+        num = num + w @ vals
+    return num / den[:, None]
+
+
+def _mut_attend_scale_d(q_rows, k, v, kept_cols, pseudo):
+    return ref.__dict__["_orig_attend"](q_rows * (1.0 / math.sqrt(q_rows.shape[-1])), k, v,
+                                        kept_cols, pseudo)
+
+
+MUTANTS = {
+    "pool divides by block size": ("pool", _mut_pool_by_blk),
+    "proxy without 1/sqrt(d)": ("proxy", _mut_proxy_unscaled),
+    "natural visit order": ("visit_order", _mut_visit_natural),
+    "diagonal block by index": ("diagonal_block", _mut_diag_index),
+    "strict threshold": ("keep_test", _mut_keep_strict),
+    "correction without n_j": ("correction_terms", _mut_corr_no_multiplicity),
+    "correction with summed value": ("correction_terms", _mut_corr_summed_value),
+    "pseudo-keys missing from denominator": ("attend_block", _mut_attend_no_pseudo_den),
+    "exact logits scaled by 1/d": ("attend_block", _mut_attend_scale_d),
+}
+
+
+@pytest.mark.parametrize("name", list(MUTANTS))
+def test_planted_mistakes_are_caught(name, monkeypatch):
+    attr, fn = MUTANTS[name]
+    monkeypatch.setitem(ref.__dict__, "_orig_attend", ref.attend_block)
+    monkeypatch.setattr(ref, attr, fn)
+    failed = []
+    for pin in PINS:
+        try:
+            pin()
+        except (AssertionError, ValueError, IndexError):
+            failed.append(pin.__name__)
+    assert failed, f"planted mistake '{name}' passed every pin"
