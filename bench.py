@@ -1,0 +1,408 @@
+#!/usr/bin/env python
+"""Benchmark of the Sol-Attn forward operator on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--config video480] [--tau 6] [--mode keep_correct] [--no-sweep]
+
+One step is one solattn_forward call (block pooling + the fused routed
+attention kernel) over one batch of synthetic spatio-temporal Q/K/V of the
+named configuration, inputs resident in HBM. The headline workload is the 480p
+video shape (B=1, H=12, N=32760, d=128, 128x128 blocks), keep_correct at tau=6.
+Prints ONE JSON line (rank 0). Multi-GPU runs are independent replicas (weak
+scaling): the operator has no cross-GPU exchange.
+
+``--impl reference`` times the fp64 CPU oracle on a bounded sample of the same
+workload on the host cores (the baseline the pages' method is checked against).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+FALLBACK_BF16_TFLOPS = 1590.0
+FALLBACK_HBM_GBS = 6650.0
+KERNEL_SOURCES = ["block_sparse_online_b200/csrc/attn_kernel.cuh", "block_sparse_online_b200/csrc/ptx_sm100.cuh",
+                  "block_sparse_online_b200/csrc/solattn_api.cu"]
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--config", default="video480")
+    ap.add_argument("--tau", type=float, default=6.0)
+    ap.add_argument("--mode", default="keep_correct", choices=["dense", "keep_drop", "keep_correct"])
+    ap.add_argument("--no-sweep", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    return ap.parse_args()
+
+
+def kernel_hash():
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            m = json.load(f)
+        return float(m["bf16_tflops"]), float(m["hbm_gbs"]), "measured"
+    return FALLBACK_BF16_TFLOPS, FALLBACK_HBM_GBS, "fallback"
+
+
+def traffic_record():
+    """DRAM bytes per attention-kernel launch from the committed ncu summary, if it was
+    taken on the current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f)
+    if rec.get("kernel_hash") != kernel_hash():
+        return None
+    return rec
+
+
+# ------------------------------------------------------------------ accounting
+
+def block_sizes(N, blk):
+    nb = -(-N // blk)
+    return np.array([min(N, (i + 1) * blk) - i * blk for i in range(nb)], dtype=np.float64)
+
+
+def executed_flops(mask_bits, N, Bq, Bk, d):
+    """4 d sum over kept (i, j) of n_i n_j: the two matmuls on the kept blocks."""
+    return 4.0 * d * float(np.einsum("bhij,i,j->", mask_bits.astype(np.float64),
+                                     block_sizes(N, Bq), block_sizes(N, Bk)))
+
+
+def unpack(mask, nKB):
+    m = mask.cpu().contiguous().numpy().view(np.uint32)
+    bits = np.unpackbits(m.view(np.uint8), bitorder="little").reshape(m.shape[:-1] + (-1,))
+    return bits[..., :nKB].astype(bool)
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, ValueError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, val in zip(names, f[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ CPU baseline (oracle)
+
+def cpu_oracle_rate(cfg, q, k, v, tau, mode, budget_s, seed=0):
+    """Time the fp64 oracle on a bounded sample and extrapolate to the whole workload.
+
+    The sample: the keep sets of one head (pooling, proxies and routing of all its
+    query blocks) plus the attention of query blocks of that head, as many as fit in
+    ``budget_s`` seconds. Returns (dense-equiv TFLOP/s, description, seconds per step).
+    """
+    import oracle.solattn_ref as ref
+    B, H, N, d = q.shape
+    nQB = -(-N // cfg.Bq)
+    rng = np.random.default_rng(seed)
+    qh, kh, vh = q[:1, :1], k[:1, :1], v[:1, :1]
+    t0 = time.perf_counter()
+    keep, _, _ = ref.keep_sets(qh, kh, cfg.Bq, cfg.Bk, tau, mode)
+    t_route = time.perf_counter() - t0
+    order = rng.permutation(nQB)
+    done, t_att = 0, 0.0
+    while done < nQB and t_att < budget_s:
+        blk = [(0, 0, int(order[done]))]
+        t1 = time.perf_counter()
+        ref.forward(qh, kh, vh, cfg.Bq, cfg.Bk, tau, mode, keep=keep, qblocks=blk)
+        t_att += time.perf_counter() - t1
+        done += 1
+    per_head = t_route + t_att / done * nQB
+    total = per_head * B * H
+    dense = cfg.dense_flops()
+    desc = (f"oracle keep sets of 1 of {B * H} heads ({t_route:.2f} s) + attention of {done} of {nQB} query "
+            f"blocks of that head ({t_att:.2f} s), extrapolated linearly to {B * H} heads x {nQB} blocks")
+    return dense / total / 1e12, desc, total
+
+
+def cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count()
+
+
+# ------------------------------------------------------------------ main
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def reference_arm(args, world, rank):
+    if rank != 0:
+        return
+    from block_sparse_online_b200 import synth
+    cfg = synth.CONFIGS[args.config]
+    q, k, v = synth.make_inputs(cfg)
+    vals, desc = [], ""
+    budget = max(2.0, min(args.cpu_seconds, 120.0 / max(1, args.steps + args.warmup)))
+    for step in range(args.warmup + args.steps):
+        rate, desc, sec = cpu_oracle_rate(cfg, q, k, v, args.tau, args.mode, budget, seed=step)
+        if step >= args.warmup:
+            vals.append(rate)
+    value = statistics.median(vals)
+    line = {
+        "impl": "reference", "metric": "sparse-attn dense-equiv TFLOP/s (fp64 CPU oracle)", "value": value,
+        "unit": "TFLOP/s (dense-equivalent)", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": cfg.dense_flops() / (value * 1e12) * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{args.config}: {cfg.note}", "tau": args.tau, "mode": args.mode},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s (dense-equivalent)", "cores": cores(), "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": "TFLOP/s (dense-equivalent)", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    world, rank, local = dist_setup(args)
+    if args.impl == "reference":
+        reference_arm(args, world, rank)
+        return
+    import torch
+    import torch.distributed as dist
+    from block_sparse_online_b200 import solattn, synth
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    cfg = synth.CONFIGS[args.config]
+    B, H, N, d = cfg.shape()
+    q, k, v = synth.make_inputs(cfg)
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    out = torch.empty_like(qd)
+    kept = torch.empty((B, H), dtype=torch.int64, device=dev)
+    ws = solattn.alloc_workspace(B, H, N, d, cfg.Bq, cfg.Bk, dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    # keep set of the headline call (for executed FLOPs); off the timed path
+    _, _, mask = solattn.solattn_forward(qd, kd, vd, cfg.Bq, cfg.Bk, args.tau, args.mode, keep_mask=True, workspace=ws)
+    st = solattn.solattn_get_status(ws)
+    if st != 0:
+        raise RuntimeError(f"device status {st}")
+    bits = unpack(mask, cfg.nKB)
+    exec_flops = executed_flops(bits, N, cfg.Bq, cfg.Bk, d)
+    dense_flops = cfg.dense_flops()
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    ka = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for _ in range(args.warmup):
+        solattn.solattn_forward(qd, kd, vd, cfg.Bq, cfg.Bk, args.tau, args.mode, out=out, kept_per_head=kept,
+                                workspace=ws)
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        solattn.solattn_forward(qd, kd, vd, cfg.Bq, cfg.Bk, args.tau, args.mode, out=out, kept_per_head=kept,
+                                workspace=ws, events=ka[i])
+        ev[i][1].record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    total_ms = t_start.elapsed_time(t_end)
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    st = solattn.solattn_get_status(ws)
+    if st != 0:
+        raise RuntimeError(f"device status {st}")
+    ms_step = total_ms / args.steps
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    attn_ms = [a.elapsed_time(b) for a, b in ka]
+    attn_avg = sum(attn_ms) / len(attn_ms)
+    value = world * dense_flops / (ms_step * 1e-3) / 1e12
+    peak_tf, peak_hbm, peak_kind = measured_peaks()
+    achieved = exec_flops / (attn_avg * 1e-3) / 1e12
+    trec = traffic_record()
+
+    # end to end through the host entry point (pinned host buffers, copies inside the timed region)
+    qh, kh, vh = q.pin_memory(), k.pin_memory(), v.pin_memory()
+    outh = torch.empty_like(q).pin_memory()
+    kh_cnt = torch.empty((B, H), dtype=torch.int64)
+    scratch = torch.empty(solattn.solattn_host_workspace_size(B, H, N, d, cfg.Bq, cfg.Bk), dtype=torch.uint8,
+                          device=dev)
+    e2e_steps = max(3, min(args.steps, 10))
+    for _ in range(2):
+        solattn.solattn_forward_host(qh, kh, vh, cfg.Bq, cfg.Bk, args.tau, args.mode, out=outh, kept_per_head=kh_cnt,
+                                     scratch=scratch)
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        solattn.solattn_forward_host(qh, kh, vh, cfg.Bq, cfg.Bk, args.tau, args.mode, out=outh, kept_per_head=kh_cnt,
+                                     scratch=scratch)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_val = world * dense_flops / (e2e_ms * 1e-3) / 1e12
+    elem = B * H * N * d
+
+    sweep = []
+    if not args.no_sweep and rank == 0:
+        for mode in ("keep_drop", "keep_correct"):
+            for tau in cfg.taus:
+                _, _, m = solattn.solattn_forward(qd, kd, vd, cfg.Bq, cfg.Bk, tau, mode, keep_mask=True, workspace=ws)
+                b = unpack(m, cfg.nKB)
+                ef = executed_flops(b, N, cfg.Bq, cfg.Bk, d)
+                ts = []
+                for i in range(8):
+                    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    a0.record(stream)
+                    solattn.solattn_forward(qd, kd, vd, cfg.Bq, cfg.Bk, tau, mode, out=out, kept_per_head=kept,
+                                            workspace=ws)
+                    a1.record(stream)
+                    torch.cuda.synchronize()
+                    if i >= 3:
+                        ts.append(a0.elapsed_time(a1))
+                ms = statistics.median(ts)
+                sweep.append({"mode": mode, "tau": None if math.isinf(tau) else tau, "ms": round(ms, 4),
+                              "keep_ratio": round(float(b.mean()), 5),
+                              "exec_tflops": round(ef / (ms * 1e-3) / 1e12, 2),
+                              "dense_equiv_tflops": round(dense_flops / (ms * 1e-3) / 1e12, 2)})
+        ts = []
+        for i in range(6):
+            a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a0.record(stream)
+            solattn.solattn_forward(qd, kd, vd, cfg.Bq, cfg.Bk, 0.0, "dense", out=out, kept_per_head=kept, workspace=ws)
+            a1.record(stream)
+            torch.cuda.synchronize()
+            if i >= 2:
+                ts.append(a0.elapsed_time(a1))
+        ms = statistics.median(ts)
+        sweep.append({"mode": "dense", "tau": None, "ms": round(ms, 4), "keep_ratio": 1.0,
+                      "exec_tflops": round(dense_flops / (ms * 1e-3) / 1e12, 2),
+                      "dense_equiv_tflops": round(dense_flops / (ms * 1e-3) / 1e12, 2)})
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, desc, _ = cpu_oracle_rate(cfg, q, k, v, args.tau, args.mode, args.cpu_seconds)
+        cpu = {"value": rate, "unit": "TFLOP/s (dense-equivalent)", "cores": cores(), "kind": "oracle",
+               "sample": desc}
+
+    if rank == 0:
+        line = {
+            "metric": "sparse-attn dense-equiv TFLOP/s (ms/call, executed TFLOP/s and keep ratio alongside)",
+            "value": round(value, 3), "unit": "TFLOP/s (dense-equivalent)", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"{args.config}: {cfg.note}", "mode": args.mode, "tau": args.tau,
+                       "B": B, "H": H, "N": N, "d": d, "Bq": cfg.Bq, "Bk": cfg.Bk,
+                       "l2": "inputs larger than L2 (q, k, v = %.0f MB)" % (3 * elem * 2 / 1e6),
+                       "parallelism": f"replicas x{world}"},
+            "keep_ratio": round(float(bits.mean()), 5),
+            "exec_tflops": round(exec_flops / (ms_step * 1e-3) / 1e12, 2),
+            "step_ms_median": round(statistics.median(step_ms), 4),
+            "attn_kernel_ms": round(attn_avg, 4),
+            "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak_tf, "unit": "TFLOP/s",
+                         "frac": round(achieved / peak_tf, 4), "peak_source": f"{peak_kind} bf16 dense (burst)",
+                         "traffic": None if trec is None else trec["dram_bytes_per_launch"],
+                         "kernel": "solattn_fwd_kernel (executed FLOPs per launch / CUDA-event duration)"},
+            "e2e": {"value": round(e2e_val, 3), "unit": "TFLOP/s (dense-equivalent)", "ms_per_step": round(e2e_ms, 3),
+                    "h2d_bytes_per_step": 3 * elem * 2, "d2h_bytes_per_step": elem * 2 + B * H * 8},
+            "gpu_launches": args.steps * (1 if args.mode == "dense" else 2),
+            "clocks": clk,
+            "cpu_baseline": cpu,
+            "sweep": sweep,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,755 @@
+// attn_kernel.cuh -- the fused Sol-Attn forward kernel for sm_100a.
+//
+// One persistent CTA per SM processes work items. An item is NT = 2 adjacent
+// 128-row query tiles of one (batch, head) pair (each tile holds 128/Bq query
+// blocks). Roles, by warp:
+//   warp 0      TMA producer: Q tiles of the item, then K_j and V_j of every key
+//               block j in the item's kept list, into a ring of shared-memory slots.
+//   warp 1      MMA issuer (one thread): S_t = Q_t K_j^T into tensor memory (TMEM),
+//               O_t += P_t V_j with P_t read from TMEM (tcgen05, bf16 -> fp32).
+//   warp 2      router: on-the-fly block thresholding and the correction sums for the
+//               NEXT item (double-buffered), from the fp32 pooled blocks in L2.
+//   warps 4..7  softmax warpgroup of tile 0, warps 8..11 of tile 1: online softmax
+//               with a lazily rescaled running max, P to TMEM, and the epilogue that
+//               merges the correction and writes bf16 rows.
+// The MMA warp interleaves the two tiles (ping-pong): while one warpgroup
+// exponentiates its S tile, the tensor core runs the other tile's P V and Q K^T.
+//
+// Method (paperlayer summary "Sol-Attn: Accelerating Video Generation Inference
+// via On-the-Fly Attention Sparsification", §3 Methodology):
+//  * routing: block proxy s = mean(Q_i) . mean(K_j) / sqrt(d) is compared, as it is
+//    produced, against the running maximum of the proxies visited so far minus tau
+//    ("On-the-fly sparsification"); key blocks are visited from query block i's
+//    diagonal block upward with wrap-around. The kept list lives only in shared
+//    memory: no proxy map and no routing indices are written to HBM.
+//  * exact attention on kept blocks with one online-softmax state per row
+//    ("Unified execution": one online-softmax state, original K/V tiles loaded only
+//    for routed indices).
+//  * each dropped block re-enters as one pseudo-key of weight n_j e^{s} and value
+//    mean(V_j) ("Approximate correction": zeroth-order proxy-score reuse with pooled
+//    keys and summed values). Because s does not depend on the query row, the
+//    correction is one d-vector and one scalar per query block, built by the router.
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <math_constants.h>
+
+#include "ptx_sm100.cuh"
+
+namespace solattn {
+
+constexpr int kMaxKeyBlocks = 1024;
+constexpr int kMaskWords = kMaxKeyBlocks / 32;
+constexpr int kStatusTimeout = -4;
+constexpr float kLog2e = 1.4426950408889634f;
+// Lazy rescaling: a row's reference max moves only when the tile max exceeds it by
+// more than this many log2 units, so P stays <= 2^8 and O is rarely rescaled.
+constexpr float kRescaleSlack = 8.0f;
+
+struct FwdParams {
+  int N;
+  int nQB;
+  int nKB;
+  int mode;  // 0 dense, 1 keep_drop, 2 keep_correct
+  float tau;
+  int items_per_head;
+  int n_items;
+  const float *qbar;  // [BH][nQB][D]
+  const float *kbar;  // [BH][nKB][D]
+  const float *vbar;  // [BH][nKB][D] (keep_correct only)
+  __nv_bfloat16 *out; // [BH][N][D]
+  unsigned long long *kept_per_head;  // [BH]
+  uint32_t *keep_mask;                // [BH][nQB][ceil(nKB/32)] or null
+  unsigned int *counter;              // work-item counter, zero at launch
+  int *status;                        // device status word
+  unsigned long long timeout_ns;      // limit of every device-side wait
+};
+
+template <int D_, int BK_, int SUBQ_, int NT_>
+struct Cfg {
+  static constexpr int D = D_;
+  static constexpr int BK = BK_;
+  static constexpr int SUBQ = SUBQ_;  // query blocks per 128-row tile
+  static constexpr int NT = NT_;      // tiles per work item
+  static constexpr int TILE_M = 128;
+  static constexpr int BQ = TILE_M / SUBQ;
+  static constexpr int NSB = NT * SUBQ;  // query blocks per work item
+  static constexpr int PANELS = D / 64;  // 128-byte swizzle panels per row
+  static constexpr int Q_TILE_BYTES = TILE_M * D * 2;
+  static constexpr int KV_BYTES = BK * D * 2;
+  static constexpr int NSLOT = (131072 / KV_BYTES) < 8 ? (131072 / KV_BYTES) : 8;
+  static constexpr int TILE_COLS = BK + D;  // TMEM columns per tile: S (aliased by P) + O
+  static constexpr int TMEM_NEED = NT * TILE_COLS;
+  static constexpr int TMEM_COLS = TMEM_NEED <= 64 ? 64 : TMEM_NEED <= 128 ? 128 : TMEM_NEED <= 256 ? 256 : 512;
+  // One control warpgroup (warp 0 producer, warp 1 MMA, warp 2 router, warp 3 spare)
+  // and one softmax warpgroup per tile. A warp may only touch TMEM lanes
+  // 32*(warp%4)..+31, so each softmax warpgroup covers the four lane quadrants once.
+  static constexpr int CTRL_WARPS = 4;
+  static constexpr int NUM_THREADS = 32 * CTRL_WARPS + 128 * NT;
+  // Register split: the control warpgroup hands registers to the softmax warpgroups,
+  // which hold a whole S row. The sum stays within the registers the block is
+  // launched with (384 threads x 168).
+  static constexpr int CTRL_REGS = 88;
+  static constexpr int SOFTMAX_REGS = 208;
+  static_assert(NT != 2 || 128 * CTRL_REGS + 256 * SOFTMAX_REGS <= 384 * 168, "register split");
+  static constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, BK, false);
+  static constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, true);
+  static_assert(TMEM_NEED <= 512, "TMEM budget");
+  static_assert(NSB <= 8, "member bits");
+};
+
+template <class C>
+struct RouteSlot {
+  int item;     // work item, or -1 when the CTA has no more work
+  int n_union;  // number of key blocks kept by at least one query block of the item
+  int pad[2];
+  float M[C::NSB];        // running proxy max (natural log units), -inf if no correction
+  float L[C::NSB];        // sum over dropped j of n_j e^{s_ij - M}
+  float Cv[C::NSB][C::D]; // sum over dropped j of n_j e^{s_ij - M} mean(V_j)
+  uint16_t jlist[kMaxKeyBlocks];  // kept key blocks (union over the item), ascending
+  uint8_t member[kMaxKeyBlocks];  // bit sb: query block sb of the item keeps jlist[u]
+};
+
+template <class C>
+struct SmemCtl {
+  RouteSlot<C> route[2];
+  uint32_t mask[C::NSB][kMaskWords];  // router scratch: keep bits per query block
+  float qrow[C::D];                    // router scratch: pooled query block
+  uint64_t full[C::NSLOT];
+  uint64_t empty[C::NSLOT];
+  uint64_t q_full, q_empty;
+  uint64_t s_full[C::NT], p_full[C::NT], o_full[C::NT], o_empty[C::NT];
+  uint64_t route_full[2], route_empty[2];
+  uint64_t mma_done;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+template <class C>
+constexpr size_t fwd_smem_bytes() {
+  return 1024 + static_cast<size_t>(C::NT) * C::Q_TILE_BYTES +
+         static_cast<size_t>(C::NSLOT) * C::KV_BYTES + sizeof(SmemCtl<C>);
+}
+
+__device__ __forceinline__ void raise_abort(int *abort_flag, int *status) {
+  atomicExch(status, kStatusTimeout);
+  *reinterpret_cast<volatile int *>(abort_flag) = 1;
+}
+
+__device__ __forceinline__ float u2f(uint32_t x) { return __uint_as_float(x); }
+
+// ------------------------------------------------------------------ router
+
+template <class C>
+__device__ __forceinline__ void route_query_block(SmemCtl<C> &sc, RouteSlot<C> &rs, const FwdParams &p,
+                                                  int bh, int sb, int qb, int lane) {
+  constexpr int D = C::D;
+  constexpr int VPL = D / 32;
+  const int nKB = p.nKB;
+  const float inv_sqrt_d = rsqrtf(static_cast<float>(D));
+  const bool correct = (p.mode == 2);
+  const int j0 = min((qb * C::BQ) / C::BK, nKB - 1);
+  const float *kb = p.kbar + static_cast<size_t>(bh) * nKB * D;
+  const float *vb = p.vbar + static_cast<size_t>(bh) * nKB * D;
+  uint32_t *msk = sc.mask[sb];
+  const float4 *qv = reinterpret_cast<const float4 *>(sc.qrow);
+
+  float M = -CUDART_INF_F;
+  float cacc[VPL];
+#pragma unroll
+  for (int e = 0; e < VPL; ++e) cacc[e] = 0.f;
+  float lacc = 0.f;
+
+  for (int t0 = 0; t0 < nKB; t0 += 32) {
+    const int tt = t0 + lane;
+    const bool valid = tt < nKB;
+    int j = j0 + tt;
+    if (j >= nKB) j -= nKB;
+    float s = -CUDART_INF_F;
+    if (valid) {
+      const float4 *kr = reinterpret_cast<const float4 *>(kb + static_cast<size_t>(j) * D);
+      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll
+      for (int c = 0; c < D / 4; ++c) {
+        const float4 kx = __ldg(kr + c);
+        const float4 qx = qv[c];
+        a0 = fmaf(qx.x, kx.x, a0);
+        a1 = fmaf(qx.y, kx.y, a1);
+        a2 = fmaf(qx.z, kx.z, a2);
+        a3 = fmaf(qx.w, kx.w, a3);
+      }
+      s = ((a0 + a1) + (a2 + a3)) * inv_sqrt_d;
+    }
+    // Running maximum in visit order: inclusive prefix max over the lanes.
+    float m = s;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const float y = __shfl_up_sync(0xffffffffu, m, off);
+      if (lane >= off) m = fmaxf(m, y);
+    }
+    m = fmaxf(m, M);
+    const bool keep = valid && (s >= m - p.tau);
+    const float Mn = __shfl_sync(0xffffffffu, m, 31);
+    if (keep) atomicOr(&msk[j >> 5], 1u << (j & 31));
+    if (correct) {
+      if (Mn > M) {
+        const float f = expf(M - Mn);  // 0 on the first chunk (M = -inf)
+#pragma unroll
+        for (int e = 0; e < VPL; ++e) cacc[e] *= f;
+        lacc *= f;
+        M = Mn;
+      }
+      const bool drop = valid && !keep;
+      const float nj = (j == nKB - 1) ? static_cast<float>(p.N - j * C::BK) : static_cast<float>(C::BK);
+      const float w = drop ? nj * expf(s - M) : 0.f;
+      lacc += w;
+      uint32_t dm = __ballot_sync(0xffffffffu, drop);
+      while (dm) {
+        const int b = __ffs(dm) - 1;
+        dm &= dm - 1;
+        const float wb = __shfl_sync(0xffffffffu, w, b);
+        const int jb = __shfl_sync(0xffffffffu, j, b);
+        const float *vr = vb + static_cast<size_t>(jb) * D + lane * VPL;
+        if constexpr (VPL == 4) {
+          const float4 vv = __ldg(reinterpret_cast<const float4 *>(vr));
+          cacc[0] = fmaf(wb, vv.x, cacc[0]);
+          cacc[1] = fmaf(wb, vv.y, cacc[1]);
+          cacc[2] = fmaf(wb, vv.z, cacc[2]);
+          cacc[3] = fmaf(wb, vv.w, cacc[3]);
+        } else {
+          const float2 vv = __ldg(reinterpret_cast<const float2 *>(vr));
+          cacc[0] = fmaf(wb, vv.x, cacc[0]);
+          cacc[1] = fmaf(wb, vv.y, cacc[1]);
+        }
+      }
+    } else {
+      M = Mn;
+    }
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) lacc += __shfl_xor_sync(0xffffffffu, lacc, off);
+#pragma unroll
+  for (int e = 0; e < VPL; ++e) rs.Cv[sb][lane * VPL + e] = correct ? cacc[e] : 0.f;
+  if (lane == 0) {
+    rs.L[sb] = correct ? lacc : 0.f;
+    rs.M[sb] = correct ? M : -CUDART_INF_F;
+  }
+}
+
+template <class C>
+__device__ void run_router(SmemCtl<C> &sc, const FwdParams &p, int lane) {
+  constexpr int D = C::D;
+  const int nKB = p.nKB;
+  const int nW = (nKB + 31) >> 5;
+  const uint32_t last_word = (nKB & 31) ? ((1u << (nKB & 31)) - 1u) : 0xffffffffu;
+  const volatile int *ab = &sc.abort_flag;
+  bool ok = true;
+  for (uint32_t r_it = 0;; ++r_it) {
+    const int s = r_it & 1;
+    bool w_ok = mbar_wait(&sc.route_empty[s], ((r_it >> 1) & 1) ^ 1, p.timeout_ns, ab);
+    if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
+    int item = 0;
+    if (lane == 0) item = static_cast<int>(atomicAdd(p.counter, 1u));
+    item = __shfl_sync(0xffffffffu, item, 0);
+    RouteSlot<C> &rs = sc.route[s];
+    if (item >= p.n_items) {
+      if (lane == 0) {
+        rs.item = -1;
+        rs.n_union = 0;
+        mbar_arrive(&sc.route_full[s]);
+      }
+      break;
+    }
+    const int bh = item / p.items_per_head;
+    const int pidx = item - bh * p.items_per_head;
+    for (int sb = 0; sb < C::NSB; ++sb)
+      for (int w = lane; w < nW; w += 32) sc.mask[sb][w] = 0u;
+    __syncwarp();
+    for (int sb = 0; sb < C::NSB; ++sb) {
+      const int qb = pidx * C::NSB + sb;
+      if (qb >= p.nQB || p.mode == 0) {
+        if (qb < p.nQB)
+          for (int w = lane; w < nW; w += 32) sc.mask[sb][w] = (w == nW - 1) ? last_word : 0xffffffffu;
+        for (int e = lane; e < D; e += 32) rs.Cv[sb][e] = 0.f;
+        if (lane == 0) {
+          rs.L[sb] = 0.f;
+          rs.M[sb] = -CUDART_INF_F;
+        }
+        continue;
+      }
+      const float *qr = p.qbar + (static_cast<size_t>(bh) * p.nQB + qb) * D;
+      for (int e = lane; e < D; e += 32) sc.qrow[e] = __ldg(qr + e);
+      __syncwarp();
+      route_query_block<C>(sc, rs, p, bh, sb, qb, lane);
+      __syncwarp();
+    }
+    // Union of the item's keep sets, ascending, with per-query-block membership bits.
+    int base = 0;
+    for (int w0 = 0; w0 < nW; w0 += 32) {
+      const int w = w0 + lane;
+      uint32_t words[C::NSB];
+      uint32_t u = 0;
+#pragma unroll
+      for (int sb = 0; sb < C::NSB; ++sb) {
+        words[sb] = (w < nW) ? sc.mask[sb][w] : 0u;
+        u |= words[sb];
+      }
+      const int cnt = __popc(u);
+      int incl = cnt;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += y;
+      }
+      int pos = base + incl - cnt;
+      while (u) {
+        const int b = __ffs(u) - 1;
+        u &= u - 1;
+        uint32_t mem = 0;
+#pragma unroll
+        for (int sb = 0; sb < C::NSB; ++sb) mem |= ((words[sb] >> b) & 1u) << sb;
+        rs.jlist[pos] = static_cast<uint16_t>(w * 32 + b);
+        rs.member[pos] = static_cast<uint8_t>(mem);
+        ++pos;
+      }
+      base += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    // Statistics: kept blocks per head, and the optional keep bit-mask.
+    unsigned long long kept = 0;
+    for (int sb = 0; sb < C::NSB; ++sb) {
+      const int qb = pidx * C::NSB + sb;
+      if (qb >= p.nQB) continue;
+      for (int w = lane; w < nW; w += 32) {
+        const uint32_t word = sc.mask[sb][w];
+        kept += __popc(word);
+        if (p.keep_mask) p.keep_mask[(static_cast<size_t>(bh) * p.nQB + qb) * nW + w] = word;
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) kept += __shfl_xor_sync(0xffffffffu, kept, off);
+    __syncwarp();
+    if (lane == 0) {
+      atomicAdd(p.kept_per_head + bh, kept);
+      rs.item = item;
+      rs.n_union = base;
+      mbar_arrive(&sc.route_full[s]);
+    }
+    __syncwarp();
+  }
+  if (!ok && lane == 0) raise_abort(&sc.abort_flag, p.status);
+}
+
+// ------------------------------------------------------------------ producer
+
+template <class C>
+__device__ void run_producer(SmemCtl<C> &sc, const FwdParams &p, uint8_t *q_smem, uint8_t *ring,
+                             const CUtensorMap *tm_q, const CUtensorMap *tm_k, const CUtensorMap *tm_v) {
+  const volatile int *ab = &sc.abort_flag;
+  uint32_t kv_it = 0, q_it = 0;
+  bool ok = true;
+  for (uint32_t r_it = 0;; ++r_it) {
+    const int s = r_it & 1;
+    if (!mbar_wait(&sc.route_full[s], (r_it >> 1) & 1, p.timeout_ns, ab)) { ok = false; break; }
+    const RouteSlot<C> &rs = sc.route[s];
+    const int item = rs.item;
+    if (item < 0) break;
+    const int bh = item / p.items_per_head;
+    const int row0 = (item - bh * p.items_per_head) * (C::NT * C::TILE_M);
+    if (!mbar_wait(&sc.q_empty, (q_it & 1) ^ 1, p.timeout_ns, ab)) { ok = false; break; }
+    mbar_arrive_expect_tx(&sc.q_full, C::NT * C::Q_TILE_BYTES);
+#pragma unroll
+    for (int t = 0; t < C::NT; ++t)
+#pragma unroll
+      for (int pn = 0; pn < C::PANELS; ++pn)
+        tma_load_3d(smem_u32(q_smem + t * C::Q_TILE_BYTES + pn * (C::TILE_M * 128)), tm_q,
+                    smem_u32(&sc.q_full), pn * 64, row0 + t * C::TILE_M, bh);
+    ++q_it;
+    const int n = rs.n_union;
+    for (int u = 0; u < n && ok; ++u) {
+      const int j = rs.jlist[u];
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const int slot = kv_it % C::NSLOT;
+        const uint32_t ph = (kv_it / C::NSLOT) & 1;
+        if (!mbar_wait(&sc.empty[slot], ph ^ 1, p.timeout_ns, ab)) { ok = false; break; }
+        mbar_arrive_expect_tx(&sc.full[slot], C::KV_BYTES);
+        uint8_t *dst = ring + slot * C::KV_BYTES;
+#pragma unroll
+        for (int pn = 0; pn < C::PANELS; ++pn)
+          tma_load_3d(smem_u32(dst + pn * (C::BK * 128)), half ? tm_v : tm_k, smem_u32(&sc.full[slot]),
+                      pn * 64, j * C::BK, bh);
+        ++kv_it;
+      }
+    }
+    if (!ok) break;
+    mbar_arrive(&sc.route_empty[s]);
+  }
+  if (!ok) raise_abort(&sc.abort_flag, p.status);
+  // No copy may outlive the block: wait (bounded, ignoring the abort flag) for the
+  // last fill of every slot and of the Q tiles to land.
+  const int zero = 0;
+  for (uint32_t f = (kv_it > C::NSLOT ? kv_it - C::NSLOT : 0); f < kv_it; ++f)
+    mbar_wait(&sc.full[f % C::NSLOT], (f / C::NSLOT) & 1, p.timeout_ns, &zero);
+  if (q_it > 0) mbar_wait(&sc.q_full, (q_it - 1) & 1, p.timeout_ns, &zero);
+}
+
+// ------------------------------------------------------------------ MMA issuer
+
+template <class C>
+__device__ __forceinline__ void issue_qk(uint32_t tmem, int t, uint32_t q_base, uint32_t k_base) {
+  const uint32_t d_tmem = tmem + t * C::TILE_COLS;
+#pragma unroll
+  for (int kk = 0; kk < C::D / 16; ++kk) {
+    const uint32_t off_q = (kk >> 2) * (C::TILE_M * 128) + (kk & 3) * 32;
+    const uint32_t off_k = (kk >> 2) * (C::BK * 128) + (kk & 3) * 32;
+    mma_bf16_ss(d_tmem, smem_desc_sw128(q_base + off_q, 16, 1024), smem_desc_sw128(k_base + off_k, 16, 1024),
+                C::IDESC_QK, kk > 0 ? 1u : 0u);
+  }
+}
+
+template <class C>
+__device__ __forceinline__ void issue_pv(uint32_t tmem, int t, uint32_t v_base, bool accumulate) {
+  const uint32_t d_tmem = tmem + t * C::TILE_COLS + C::BK;
+  const uint32_t p_tmem = tmem + t * C::TILE_COLS;
+#pragma unroll
+  for (int kk = 0; kk < C::BK / 16; ++kk) {
+    mma_bf16_ts(d_tmem, p_tmem + kk * 8, smem_desc_sw128(v_base + kk * (16 * 128), C::BK * 128, 1024),
+                C::IDESC_PV, (accumulate || kk > 0) ? 1u : 0u);
+  }
+}
+
+template <class C>
+__device__ void run_mma(SmemCtl<C> &sc, const FwdParams &p, uint32_t tmem, uint8_t *q_smem, uint8_t *ring) {
+  const volatile int *ab = &sc.abort_flag;
+  const uint32_t q_base = smem_u32(q_smem);
+  const uint32_t ring_base = smem_u32(ring);
+  constexpr uint32_t TILE_BITS = (1u << C::SUBQ) - 1u;
+  uint32_t kv_it = 0, q_it = 0, o_it = 0;
+  uint32_t p_ph[C::NT];
+#pragma unroll
+  for (int t = 0; t < C::NT; ++t) p_ph[t] = 0;
+  bool ok = true;
+  auto wait = [&](uint64_t *bar, uint32_t par) {
+    if (!ok) return false;
+    if (!mbar_wait(bar, par, p.timeout_ns, ab)) ok = false;
+    else tc_fence_after_sync();
+    return ok;
+  };
+  for (uint32_t r_it = 0; ok; ++r_it) {
+    const int s = r_it & 1;
+    if (!wait(&sc.route_full[s], (r_it >> 1) & 1)) break;
+    const RouteSlot<C> &rs = sc.route[s];
+    const int item = rs.item;
+    if (item < 0) break;
+    const int n = rs.n_union;
+    if (!wait(&sc.q_full, q_it & 1)) break;
+    ++q_it;
+    // prologue: S for the first kept key block
+    int kslot = kv_it % C::NSLOT;
+    if (!wait(&sc.full[kslot], (kv_it / C::NSLOT) & 1)) break;
+    ++kv_it;
+    uint32_t mem = rs.member[0];
+#pragma unroll
+    for (int t = 0; t < C::NT; ++t)
+      if ((mem >> (t * C::SUBQ)) & TILE_BITS) {
+        issue_qk<C>(tmem, t, q_base + t * C::Q_TILE_BYTES, ring_base + kslot * C::KV_BYTES);
+        tc_commit(&sc.s_full[t]);
+      }
+    tc_commit(&sc.empty[kslot]);
+    if (n == 1) tc_commit(&sc.q_empty);
+    bool first[C::NT];
+#pragma unroll
+    for (int t = 0; t < C::NT; ++t) first[t] = true;
+    for (int u = 0; u < n && ok; ++u) {
+      const int vslot = kv_it % C::NSLOT;
+      if (!wait(&sc.full[vslot], (kv_it / C::NSLOT) & 1)) break;
+      ++kv_it;
+      const bool has_next = (u + 1) < n;
+      uint32_t memn = 0;
+      if (has_next) {
+        kslot = kv_it % C::NSLOT;
+        if (!wait(&sc.full[kslot], (kv_it / C::NSLOT) & 1)) break;
+        ++kv_it;
+        memn = rs.member[u + 1];
+      }
+#pragma unroll
+      for (int t = 0; t < C::NT; ++t) {
+        if ((mem >> (t * C::SUBQ)) & TILE_BITS) {
+          if (!wait(&sc.p_full[t], p_ph[t])) break;
+          p_ph[t] ^= 1;
+          if (first[t] && !wait(&sc.o_empty[t], (o_it & 1) ^ 1)) break;
+          issue_pv<C>(tmem, t, ring_base + vslot * C::KV_BYTES, !first[t]);
+          first[t] = false;
+        }
+        if ((memn >> (t * C::SUBQ)) & TILE_BITS) {
+          issue_qk<C>(tmem, t, q_base + t * C::Q_TILE_BYTES, ring_base + kslot * C::KV_BYTES);
+          tc_commit(&sc.s_full[t]);
+        }
+      }
+      if (!ok) break;
+      tc_commit(&sc.empty[vslot]);
+      if (has_next) {
+        tc_commit(&sc.empty[kslot]);
+        if (u + 2 == n) tc_commit(&sc.q_empty);
+      }
+      mem = memn;
+    }
+    if (!ok) break;
+#pragma unroll
+    for (int t = 0; t < C::NT; ++t) {
+      if (first[t] && !wait(&sc.o_empty[t], (o_it & 1) ^ 1)) break;
+      tc_commit(&sc.o_full[t]);
+    }
+    if (!ok) break;
+    ++o_it;
+    mbar_arrive(&sc.route_empty[s]);
+  }
+  if (!ok) raise_abort(&sc.abort_flag, p.status);
+  // Every tcgen05 operation issued here must finish before TMEM is released.
+  const int zero = 0;
+  tc_commit(&sc.mma_done);
+  mbar_wait(&sc.mma_done, 0, p.timeout_ns, &zero);
+}
+
+// ------------------------------------------------------------------ softmax / epilogue
+
+template <class C>
+__device__ void run_softmax(SmemCtl<C> &sc, const FwdParams &p, uint32_t tmem, int t, int warp, int lane) {
+  constexpr int BK = C::BK;
+  constexpr int D = C::D;
+  constexpr uint32_t TILE_BITS = ((1u << C::SUBQ) - 1u);
+  const volatile int *ab = &sc.abort_flag;
+  const int wq = warp & 3;  // TMEM lane quadrant this warp may access
+  const int row = wq * 32 + lane;
+  const uint32_t s_addr = tmem + (static_cast<uint32_t>(wq * 32) << 16) + t * C::TILE_COLS;
+  const uint32_t o_addr = s_addr + BK;
+  const float sc_log2 = kLog2e * rsqrtf(static_cast<float>(D));
+  const int sb = t * C::SUBQ + (C::SUBQ == 2 ? (row >> 6) : 0);
+  const uint32_t row_bit = 1u << sb;
+  const uint32_t tile_bits = TILE_BITS << (t * C::SUBQ);
+  uint32_t s_ph = 0;
+  bool ok = true;
+  auto wait = [&](uint64_t *bar, uint32_t par) {
+    bool w = mbar_wait(bar, par, p.timeout_ns, ab);
+    w = __all_sync(0xffffffffu, w);
+    if (!w) ok = false;
+    else tc_fence_after_sync();
+    return w;
+  };
+  for (uint32_t r_it = 0; ok; ++r_it) {
+    const int s = r_it & 1;
+    if (!wait(&sc.route_full[s], (r_it >> 1) & 1)) break;
+    const RouteSlot<C> &rs = sc.route[s];
+    const int item = rs.item;
+    if (item < 0) break;
+    const int bh = item / p.items_per_head;
+    const int pidx = item - bh * p.items_per_head;
+    const int grow = pidx * (C::NT * C::TILE_M) + t * C::TILE_M + row;
+    const int n = rs.n_union;
+    float m_ref = -CUDART_INF_F;  // reference max of this row, log2 units
+    float l = 0.f;
+    bool any = false;
+    for (int u = 0; u < n; ++u) {
+      const uint32_t mem = rs.member[u];
+      if (!(mem & tile_bits)) continue;
+      const int j = rs.jlist[u];
+      if (!wait(&sc.s_full[t], s_ph)) break;
+      s_ph ^= 1;
+      uint32_t sr[BK / 32][32];
+#pragma unroll
+      for (int c = 0; c < BK / 32; ++c) tmem_ld32(s_addr + c * 32, sr[c]);
+      tmem_wait_ld();
+#pragma unroll
+      for (int c = 0; c < BK / 32; ++c) reg_fence32(sr[c]);
+      const bool rk = (mem & row_bit) != 0;
+      const int ncol = (j == p.nKB - 1) ? (p.N - j * BK) : BK;
+      float mx = -CUDART_INF_F;
+      if (rk) {
+#pragma unroll
+        for (int c = 0; c < BK / 32; ++c)
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            if (c * 32 + e < ncol) mx = fmaxf(mx, u2f(sr[c][e]));
+      }
+      const float mxs = mx * sc_log2;
+      float alpha = 1.f;
+      bool resc = false;
+      if (mxs > m_ref + kRescaleSlack) {
+        if (m_ref != -CUDART_INF_F) {
+          alpha = ex2_approx(m_ref - mxs);
+          resc = true;
+        }
+        m_ref = mxs;
+      }
+      l *= alpha;
+      const float neg_m = (m_ref == -CUDART_INF_F) ? 0.f : -m_ref;
+      float lsum = 0.f;
+#pragma unroll
+      for (int h = 0; h < BK / 64; ++h) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int col = h * 64 + 2 * e;
+          const float x0 = u2f(sr[col >> 5][col & 31]);
+          const float x1 = u2f(sr[(col + 1) >> 5][(col + 1) & 31]);
+          const float p0 = (rk && col < ncol) ? ex2_approx(fmaf(x0, sc_log2, neg_m)) : 0.f;
+          const float p1 = (rk && col + 1 < ncol) ? ex2_approx(fmaf(x1, sc_log2, neg_m)) : 0.f;
+          lsum += p0 + p1;
+          pk[e] = pack_bf16x2(p0, p1);
+        }
+        tmem_st32(s_addr + h * 32, pk);
+      }
+      l += lsum;
+      if (__any_sync(0xffffffffu, resc)) {
+        // The previous P V of this tile has completed (the commit that signalled this
+        // S tile was issued after it), so O can be rescaled in place before the next one.
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(o_addr + c * 32, o);
+          tmem_wait_ld();
+          reg_fence32(o);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(u2f(o[e]) * alpha);
+          tmem_st32(o_addr + c * 32, o);
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before_sync();
+      mbar_arrive(&sc.p_full[t]);
+      any = true;
+    }
+    if (!ok) break;
+    // Epilogue: O / l merged with the correction of this row's query block.
+    if (!wait(&sc.o_full[t], r_it & 1)) break;
+    if (any) {
+      const int qb = pidx * C::NSB + sb;
+      const bool valid = (grow < p.N) && (qb < p.nQB);
+      float a = 1.f, b = 0.f;
+      const float Lc = rs.L[sb];
+      if (Lc > 0.f) {
+        const float M2 = rs.M[sb] * kLog2e;
+        const float Ms = fmaxf(m_ref, M2);
+        a = ex2_approx(m_ref - Ms);
+        b = ex2_approx(M2 - Ms);
+      }
+      const float inv = 1.f / (a * l + b * Lc);
+      const float *cv = rs.Cv[sb];
+      uint4 *dst = reinterpret_cast<uint4 *>(p.out + (static_cast<size_t>(bh) * p.N + grow) * D);
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t o[32];
+        tmem_ld32(o_addr + c * 32, o);
+        tmem_wait_ld();
+        reg_fence32(o);
+        if (valid) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float y0 = fmaf(a, u2f(o[2 * e]), b * cv[c * 32 + 2 * e]) * inv;
+            const float y1 = fmaf(a, u2f(o[2 * e + 1]), b * cv[c * 32 + 2 * e + 1]) * inv;
+            pk[e] = pack_bf16x2(y0, y1);
+          }
+#pragma unroll
+          for (int v = 0; v < 4; ++v)
+            dst[c * 4 + v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+        }
+      }
+    }
+    tc_fence_before_sync();
+    mbar_arrive(&sc.o_empty[t]);
+    mbar_arrive(&sc.route_empty[s]);
+  }
+  if (!ok && lane == 0) raise_abort(&sc.abort_flag, p.status);
+}
+
+// ------------------------------------------------------------------ kernel
+
+template <class C>
+__global__ void __launch_bounds__(C::NUM_THREADS, 1)
+    solattn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                       const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *q_smem = base;
+  uint8_t *ring = base + C::NT * C::Q_TILE_BYTES;
+  SmemCtl<C> &sc = *reinterpret_cast<SmemCtl<C> *>(ring + C::NSLOT * C::KV_BYTES);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::NSLOT; ++i) {
+      mbar_init(&sc.full[i], 1);
+      mbar_init(&sc.empty[i], 1);
+    }
+    mbar_init(&sc.q_full, 1);
+    mbar_init(&sc.q_empty, 1);
+    for (int t = 0; t < C::NT; ++t) {
+      mbar_init(&sc.s_full[t], 1);
+      mbar_init(&sc.p_full[t], 128);
+      mbar_init(&sc.o_full[t], 1);
+      mbar_init(&sc.o_empty[t], 128);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&sc.route_full[s], 1);
+      mbar_init(&sc.route_empty[s], 2 + 128 * C::NT);
+    }
+    mbar_init(&sc.mma_done, 1);
+    sc.abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+  }
+  if (warp == 1) {
+    tmem_alloc(&sc.tmem_base, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem = sc.tmem_base;
+
+  if (warp < C::CTRL_WARPS) {
+    regs_dec<C::CTRL_REGS>();
+    if (warp == 0) {
+      if (lane == 0) run_producer<C>(sc, p, q_smem, ring, &tm_q, &tm_k, &tm_v);
+    } else if (warp == 1) {
+      if (lane == 0) run_mma<C>(sc, p, tmem, q_smem, ring);
+    } else if (warp == 2) {
+      run_router<C>(sc, p, lane);
+    }
+  } else {
+    regs_inc<C::SOFTMAX_REGS>();
+    run_softmax<C>(sc, p, tmem, (warp - C::CTRL_WARPS) >> 2, warp, lane);
+  }
+
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after_sync();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// Device watchdog self-test: one thread waits on a barrier that nobody completes.
+__global__ void watchdog_selftest_kernel(int *status, unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const bool ok = mbar_wait(&bar, 0, limit_ns, &abort_flag);
+    *status = ok ? 0 : kStatusTimeout;
+  }
+}
+
+}  // namespace solattn

@@ -1,0 +1,345 @@
+// solattn_api.cu -- host side of libsolattn: argument checks, workspace layout,
+// TMA descriptors and kernel launches behind the C ABI declared in solattn.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "attn_kernel.cuh"
+#include "pool_kernel.cuh"
+#include "solattn.h"
+
+namespace {
+
+using namespace solattn;
+
+constexpr size_t kAlign = 256;
+constexpr size_t kHeaderBytes = 256;  // [0]: work counter (u32), [4]: status word (i32)
+constexpr unsigned long long kDefaultTimeoutNs = 2000000000ull;  // 2 s per device-side wait
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+int nblocks(int N, int blk) { return (N + blk - 1) / blk; }
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+struct WsLayout {
+  size_t qbar, kbar, vbar, total;
+};
+
+int check_shape(int B, int H, int N, int d, int Bq, int Bk) {
+  if (B < 1 || H < 1 || N < 1) return SOLATTN_EINVAL;
+  if (d != 64 && d != 128) return SOLATTN_EUNSUPPORTED;
+  if ((Bq != 64 && Bq != 128) || (Bk != 64 && Bk != 128)) return SOLATTN_EUNSUPPORTED;
+  if (nblocks(N, Bk) > SOLATTN_MAX_KEY_BLOCKS) return SOLATTN_EUNSUPPORTED;
+  if (static_cast<long long>(B) * H > 65535) return SOLATTN_EUNSUPPORTED;  // pooling grid y
+  return SOLATTN_OK;
+}
+
+WsLayout ws_layout(int B, int H, int N, int d, int Bq, int Bk) {
+  const size_t bh = static_cast<size_t>(B) * H;
+  WsLayout w;
+  w.qbar = kHeaderBytes;
+  w.kbar = w.qbar + align_up(bh * nblocks(N, Bq) * d * sizeof(float), kAlign);
+  w.vbar = w.kbar + align_up(bh * nblocks(N, Bk) * d * sizeof(float), kAlign);
+  w.total = w.vbar + align_up(bh * nblocks(N, Bk) * d * sizeof(float), kAlign);
+  return w;
+}
+
+struct DeviceInfo {
+  int sms = 0;
+  int major = 0;
+  bool known = false;
+};
+
+std::mutex g_mu;
+DeviceInfo g_dev[64];
+
+int device_info(DeviceInfo *out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return SOLATTN_ECUDA;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_dev[dev].known) {
+    int sms = 0, major = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return SOLATTN_ECUDA;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return SOLATTN_ECUDA;
+    g_dev[dev].sms = sms;
+    g_dev[dev].major = major;
+    g_dev[dev].known = true;
+  }
+  *out = g_dev[dev];
+  return SOLATTN_OK;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// 3-D view (d, N, B*H) of a contiguous bf16 [B][H][N][d] tensor; boxes of 64 x rows x 1
+// with the 128-byte swizzle. Rows past N read as zeros.
+int make_map(CUtensorMap *map, const void *ptr, int d, int N, int BH, int box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return SOLATTN_ECUDA;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(N) * d * 2};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? SOLATTN_OK : SOLATTN_ECUDA;
+}
+
+int launch_pool(const PoolArgs &args, int BH, int d, int max_nb, cudaStream_t st) {
+  dim3 grid(max_nb, BH, args.njobs);
+  if (d == 128)
+    pool_kernel<128><<<grid, 128, 0, st>>>(args);
+  else
+    pool_kernel<64><<<grid, 128, 0, st>>>(args);
+  return cudaGetLastError() == cudaSuccess ? SOLATTN_OK : SOLATTN_ECUDA;
+}
+
+template <class C>
+int launch_fwd(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv, const FwdParams &p, int sms,
+               cudaStream_t st) {
+  constexpr size_t smem = fwd_smem_bytes<C>();
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return SOLATTN_ECUDA;
+  if (!attr_set[dev]) {
+    if (cudaFuncSetAttribute(solattn_fwd_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+      return SOLATTN_ECUDA;
+    attr_set[dev] = true;
+  }
+  const int grid = p.n_items < sms ? p.n_items : sms;
+  solattn_fwd_kernel<C><<<grid, C::NUM_THREADS, smem, st>>>(mq, mk, mv, p);
+  return cudaGetLastError() == cudaSuccess ? SOLATTN_OK : SOLATTN_ECUDA;
+}
+
+template <int D, int BK, int SUBQ>
+int dispatch_tiles(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv, FwdParams p, int sms,
+                   cudaStream_t st) {
+  using C = Cfg<D, BK, SUBQ, 2>;
+  p.items_per_head = (p.N + C::NT * C::TILE_M - 1) / (C::NT * C::TILE_M);
+  return launch_fwd<C>(mq, mk, mv, p, sms, st);
+}
+
+int dispatch(int d, int Bq, int Bk, const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
+             const FwdParams &p, int sms, cudaStream_t st) {
+  const int subq = 128 / Bq;
+  if (d == 128) {
+    if (Bk == 128) return subq == 1 ? dispatch_tiles<128, 128, 1>(mq, mk, mv, p, sms, st)
+                                    : dispatch_tiles<128, 128, 2>(mq, mk, mv, p, sms, st);
+    return subq == 1 ? dispatch_tiles<128, 64, 1>(mq, mk, mv, p, sms, st)
+                     : dispatch_tiles<128, 64, 2>(mq, mk, mv, p, sms, st);
+  }
+  if (Bk == 128) return subq == 1 ? dispatch_tiles<64, 128, 1>(mq, mk, mv, p, sms, st)
+                                  : dispatch_tiles<64, 128, 2>(mq, mk, mv, p, sms, st);
+  return subq == 1 ? dispatch_tiles<64, 64, 1>(mq, mk, mv, p, sms, st)
+                   : dispatch_tiles<64, 64, 2>(mq, mk, mv, p, sms, st);
+}
+
+int items_total(int B, int H, int N) {
+  // Both tile shapes cover 2 x 128 query rows per work item.
+  return B * H * ((N + 255) / 256);
+}
+
+int forward_impl(const void *q, const void *k, const void *v, void *out, int B, int H, int N, int d, int Bq, int Bk,
+                 float tau, int mode, const solattn_stats *stats, void *workspace, size_t ws_bytes, void *stream,
+                 void *ev_attn_begin, void *ev_attn_end) {
+  if (!q || !k || !v || !out || !stats || !stats->kept_per_head) return SOLATTN_EINVAL;
+  const int rc = check_shape(B, H, N, d, Bq, Bk);
+  if (rc != SOLATTN_OK) return rc;
+  if (mode < SOLATTN_DENSE || mode > SOLATTN_KEEP_CORRECT) return SOLATTN_EINVAL;
+  if (!(tau >= 0.f)) return SOLATTN_EINVAL;  // negative or NaN
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16)) return SOLATTN_EINVAL;
+  if (!aligned(stats->kept_per_head, 8) || (stats->keep_mask && !aligned(stats->keep_mask, 4)))
+    return SOLATTN_EINVAL;
+  const WsLayout wl = ws_layout(B, H, N, d, Bq, Bk);
+  if (!workspace || !aligned(workspace, kAlign) || ws_bytes < wl.total) return SOLATTN_EWORKSPACE;
+  DeviceInfo di;
+  if (device_info(&di) != SOLATTN_OK) return SOLATTN_ECUDA;
+  if (di.major != 10) return SOLATTN_EUNSUPPORTED;
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  const int BH = B * H;
+  const int nQB = nblocks(N, Bq), nKB = nblocks(N, Bk);
+  float *qbar = reinterpret_cast<float *>(ws + wl.qbar);
+  float *kbar = reinterpret_cast<float *>(ws + wl.kbar);
+  float *vbar = reinterpret_cast<float *>(ws + wl.vbar);
+
+  CUtensorMap mq, mk, mv;
+  if (make_map(&mq, q, d, N, BH, 128) != SOLATTN_OK || make_map(&mk, k, d, N, BH, Bk) != SOLATTN_OK ||
+      make_map(&mv, v, d, N, BH, Bk) != SOLATTN_OK)
+    return SOLATTN_ECUDA;
+
+  if (cudaMemsetAsync(ws, 0, kHeaderBytes, st) != cudaSuccess) return SOLATTN_ECUDA;
+  if (cudaMemsetAsync(stats->kept_per_head, 0, sizeof(int64_t) * BH, st) != cudaSuccess) return SOLATTN_ECUDA;
+
+  if (mode != SOLATTN_DENSE) {
+    PoolArgs a{};
+    a.job[0] = PoolJob{static_cast<const __nv_bfloat16 *>(q), qbar, Bq, nQB};
+    a.job[1] = PoolJob{static_cast<const __nv_bfloat16 *>(k), kbar, Bk, nKB};
+    a.job[2] = PoolJob{static_cast<const __nv_bfloat16 *>(v), vbar, Bk, nKB};
+    a.njobs = (mode == SOLATTN_KEEP_CORRECT) ? 3 : 2;
+    a.N = N;
+    const int rcp = launch_pool(a, BH, d, nQB > nKB ? nQB : nKB, st);
+    if (rcp != SOLATTN_OK) return rcp;
+  }
+
+  FwdParams p{};
+  p.N = N;
+  p.nQB = nQB;
+  p.nKB = nKB;
+  p.mode = mode;
+  p.tau = tau;
+  p.n_items = items_total(B, H, N);
+  p.qbar = qbar;
+  p.kbar = kbar;
+  p.vbar = vbar;
+  p.out = static_cast<__nv_bfloat16 *>(out);
+  p.kept_per_head = reinterpret_cast<unsigned long long *>(stats->kept_per_head);
+  p.keep_mask = stats->keep_mask;
+  p.counter = reinterpret_cast<unsigned int *>(ws);
+  p.status = reinterpret_cast<int *>(ws + 4);
+  p.timeout_ns = kDefaultTimeoutNs;
+  if (ev_attn_begin && cudaEventRecord(static_cast<cudaEvent_t>(ev_attn_begin), st) != cudaSuccess)
+    return SOLATTN_ECUDA;
+  const int rl = dispatch(d, Bq, Bk, mq, mk, mv, p, di.sms, st);
+  if (rl != SOLATTN_OK) return rl;
+  if (ev_attn_end && cudaEventRecord(static_cast<cudaEvent_t>(ev_attn_end), st) != cudaSuccess)
+    return SOLATTN_ECUDA;
+  return SOLATTN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t solattn_workspace_size(int B, int H, int N, int d, int Bq, int Bk) {
+  if (check_shape(B, H, N, d, Bq, Bk) != SOLATTN_OK) return 0;
+  return ws_layout(B, H, N, d, Bq, Bk).total;
+}
+
+int solattn_pool(const void *x, float *xbar, int B, int H, int N, int d, int blk, void *stream) {
+  if (!x || !xbar) return SOLATTN_EINVAL;
+  const int rc = check_shape(B, H, N, d, blk, blk);
+  if (rc != SOLATTN_OK) return rc;
+  if (!aligned(x, 16) || !aligned(xbar, 16)) return SOLATTN_EINVAL;
+  DeviceInfo di;
+  if (device_info(&di) != SOLATTN_OK) return SOLATTN_ECUDA;
+  if (di.major != 10) return SOLATTN_EUNSUPPORTED;
+  PoolArgs a{};
+  a.job[0] = PoolJob{static_cast<const __nv_bfloat16 *>(x), xbar, blk, nblocks(N, blk)};
+  a.njobs = 1;
+  a.N = N;
+  return launch_pool(a, B * H, d, nblocks(N, blk), static_cast<cudaStream_t>(stream));
+}
+
+int solattn_forward(const void *q, const void *k, const void *v, void *out, int B, int H, int N, int d, int Bq,
+                    int Bk, float tau, int mode, const solattn_stats *stats, void *workspace, size_t ws_bytes,
+                    void *stream) {
+  return forward_impl(q, k, v, out, B, H, N, d, Bq, Bk, tau, mode, stats, workspace, ws_bytes, stream, nullptr,
+                      nullptr);
+}
+
+int solattn_forward_events(const void *q, const void *k, const void *v, void *out, int B, int H, int N, int d,
+                           int Bq, int Bk, float tau, int mode, const solattn_stats *stats, void *workspace,
+                           size_t ws_bytes, void *stream, void *ev_attn_begin, void *ev_attn_end) {
+  return forward_impl(q, k, v, out, B, H, N, d, Bq, Bk, tau, mode, stats, workspace, ws_bytes, stream,
+                      ev_attn_begin, ev_attn_end);
+}
+
+int solattn_get_status(const void *workspace, void *stream) {
+  if (!workspace) return SOLATTN_EWORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int status = 0;
+  if (cudaMemcpyAsync(&status, static_cast<const uint8_t *>(workspace) + 4, sizeof(int), cudaMemcpyDeviceToHost,
+                      st) != cudaSuccess)
+    return SOLATTN_ECUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return SOLATTN_ECUDA;
+  return status;
+}
+
+size_t solattn_host_workspace_size(int B, int H, int N, int d, int Bq, int Bk) {
+  if (check_shape(B, H, N, d, Bq, Bk) != SOLATTN_OK) return 0;
+  const size_t elems = static_cast<size_t>(B) * H * N * d;
+  const size_t t = align_up(elems * 2, kAlign);
+  const size_t kp = align_up(sizeof(int64_t) * B * H, kAlign);
+  return 4 * t + kp + ws_layout(B, H, N, d, Bq, Bk).total;
+}
+
+int solattn_forward_host(const void *q, const void *k, const void *v, void *out, int B, int H, int N, int d,
+                         int Bq, int Bk, float tau, int mode, int64_t *kept_per_head, void *dev_scratch,
+                         size_t scratch_bytes, void *stream) {
+  if (!q || !k || !v || !out) return SOLATTN_EINVAL;
+  const int rc = check_shape(B, H, N, d, Bq, Bk);
+  if (rc != SOLATTN_OK) return rc;
+  const size_t need = solattn_host_workspace_size(B, H, N, d, Bq, Bk);
+  if (!dev_scratch || !aligned(dev_scratch, kAlign) || scratch_bytes < need) return SOLATTN_EWORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t bytes = static_cast<size_t>(B) * H * N * d * 2;
+  const size_t t = align_up(bytes, kAlign);
+  uint8_t *base = static_cast<uint8_t *>(dev_scratch);
+  uint8_t *dq = base, *dk = base + t, *dv = base + 2 * t, *dout = base + 3 * t;
+  int64_t *dkept = reinterpret_cast<int64_t *>(base + 4 * t);
+  uint8_t *ws = base + 4 * t + align_up(sizeof(int64_t) * B * H, kAlign);
+  const size_t ws_bytes = scratch_bytes - (ws - base);
+  if (cudaMemcpyAsync(dq, q, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+      cudaMemcpyAsync(dk, k, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+      cudaMemcpyAsync(dv, v, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess)
+    return SOLATTN_ECUDA;
+  solattn_stats stats{dkept, nullptr};
+  const int rf = solattn_forward(dq, dk, dv, dout, B, H, N, d, Bq, Bk, tau, mode, &stats, ws, ws_bytes, stream);
+  if (rf != SOLATTN_OK) return rf;
+  if (cudaMemcpyAsync(out, dout, bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess) return SOLATTN_ECUDA;
+  if (kept_per_head &&
+      cudaMemcpyAsync(kept_per_head, dkept, sizeof(int64_t) * B * H, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return SOLATTN_ECUDA;
+  return solattn_get_status(ws, stream);
+}
+
+int solattn_watchdog_selftest(void *workspace, size_t ws_bytes, uint64_t limit_ns, void *stream) {
+  if (!workspace || !aligned(workspace, kAlign) || ws_bytes < kHeaderBytes) return SOLATTN_EWORKSPACE;
+  DeviceInfo di;
+  if (device_info(&di) != SOLATTN_OK) return SOLATTN_ECUDA;
+  if (di.major != 10) return SOLATTN_EUNSUPPORTED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int *status = reinterpret_cast<int *>(static_cast<uint8_t *>(workspace) + 4);
+  if (cudaMemsetAsync(workspace, 0, kHeaderBytes, st) != cudaSuccess) return SOLATTN_ECUDA;
+  watchdog_selftest_kernel<<<1, 32, 0, st>>>(status, static_cast<unsigned long long>(limit_ns));
+  return cudaGetLastError() == cudaSuccess ? SOLATTN_OK : SOLATTN_ECUDA;
+}
+
+const char *solattn_strerror(int status) {
+  switch (status) {
+    case SOLATTN_OK: return "ok";
+    case SOLATTN_EINVAL: return "invalid argument";
+    case SOLATTN_EUNSUPPORTED: return "unsupported shape or device";
+    case SOLATTN_ECUDA: return "CUDA error";
+    case SOLATTN_ETIMEOUT: return "device-side wait timed out";
+    case SOLATTN_EWORKSPACE: return "workspace missing, misaligned or too small";
+    default: return "unknown status";
+  }
+}
+
+}  // extern "C"

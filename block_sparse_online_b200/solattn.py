@@ -1,0 +1,212 @@
+"""ctypes binding of libsolattn (the C ABI in include/solattn.h).
+
+Argument marshalling only: every step of the operator runs in the library's
+CUDA kernels. PyTorch supplies device memory and the current stream. Loading
+fails loudly if ``libsolattn.so`` has not been built; there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsolattn.so")
+
+SOLATTN_DENSE = 0
+SOLATTN_KEEP_DROP = 1
+SOLATTN_KEEP_CORRECT = 2
+MODES = {"dense": SOLATTN_DENSE, "keep_drop": SOLATTN_KEEP_DROP, "keep_correct": SOLATTN_KEEP_CORRECT}
+
+SOLATTN_OK = 0
+SOLATTN_EINVAL = -1
+SOLATTN_EUNSUPPORTED = -2
+SOLATTN_ECUDA = -3
+SOLATTN_ETIMEOUT = -4
+SOLATTN_EWORKSPACE = -5
+MAX_KEY_BLOCKS = 1024
+
+EXPORTS = ("solattn_workspace_size", "solattn_pool", "solattn_forward", "solattn_forward_events",
+           "solattn_get_status",
+           "solattn_host_workspace_size", "solattn_forward_host", "solattn_watchdog_selftest",
+           "solattn_strerror")
+
+
+class SolAttnError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {strerror(status)} ({status})")
+        self.status = status
+
+
+class _Stats(ctypes.Structure):
+    _fields_ = [("kept_per_head", ctypes.c_void_p), ("keep_mask", ctypes.c_void_p)]
+
+
+def _load():
+    if not os.path.exists(_LIB_PATH):
+        raise ImportError(f"libsolattn.so is not built ({_LIB_PATH}); run "
+                          "`python -m block_sparse_online_b200.build`")
+    lib = ctypes.CDLL(_LIB_PATH)
+    i, sz, vp, f = ctypes.c_int, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_float
+    lib.solattn_workspace_size.argtypes = [i, i, i, i, i, i]
+    lib.solattn_workspace_size.restype = sz
+    lib.solattn_host_workspace_size.argtypes = [i, i, i, i, i, i]
+    lib.solattn_host_workspace_size.restype = sz
+    lib.solattn_pool.argtypes = [vp, vp, i, i, i, i, i, vp]
+    lib.solattn_pool.restype = i
+    lib.solattn_forward.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, f, i, ctypes.POINTER(_Stats), vp, sz, vp]
+    lib.solattn_forward.restype = i
+    lib.solattn_forward_events.argtypes = lib.solattn_forward.argtypes + [vp, vp]
+    lib.solattn_forward_events.restype = i
+    lib.solattn_forward_host.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp, vp, sz, vp]
+    lib.solattn_forward_host.restype = i
+    lib.solattn_get_status.argtypes = [vp, vp]
+    lib.solattn_get_status.restype = i
+    lib.solattn_watchdog_selftest.argtypes = [vp, sz, ctypes.c_uint64, vp]
+    lib.solattn_watchdog_selftest.restype = i
+    lib.solattn_strerror.argtypes = [i]
+    lib.solattn_strerror.restype = ctypes.c_char_p
+    return lib
+
+
+_lib = _load()
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def strerror(status: int) -> str:
+    return _lib.solattn_strerror(int(status)).decode()
+
+
+def _check(status: int, what: str):
+    if status != SOLATTN_OK:
+        raise SolAttnError(status, what)
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _mode(mode) -> int:
+    return MODES[mode] if isinstance(mode, str) else int(mode)
+
+
+def _bhnd(x: torch.Tensor):
+    if x.dim() != 4:
+        raise ValueError("expected a [B, H, N, d] tensor")
+    return tuple(int(s) for s in x.shape)
+
+
+def solattn_workspace_size(B, H, N, d, Bq, Bk) -> int:
+    return int(_lib.solattn_workspace_size(B, H, N, d, Bq, Bk))
+
+
+def solattn_host_workspace_size(B, H, N, d, Bq, Bk) -> int:
+    return int(_lib.solattn_host_workspace_size(B, H, N, d, Bq, Bk))
+
+
+def alloc_workspace(B, H, N, d, Bq, Bk, device="cuda") -> torch.Tensor:
+    n = solattn_workspace_size(B, H, N, d, Bq, Bk)
+    if n == 0:
+        raise SolAttnError(SOLATTN_EUNSUPPORTED, "solattn_workspace_size")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def solattn_pool(x: torch.Tensor, blk: int, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Block means of a bf16 [B, H, N, d] CUDA tensor -> fp32 [B, H, ceil(N/blk), d]."""
+    B, H, N, d = _bhnd(x)
+    if x.dtype != torch.bfloat16 or not x.is_cuda or not x.is_contiguous():
+        raise ValueError("x must be a contiguous bf16 CUDA tensor")
+    nb = -(-N // blk)
+    if out is None:
+        out = torch.empty((B, H, nb, d), dtype=torch.float32, device=x.device)
+    _check(_lib.solattn_pool(x.data_ptr(), out.data_ptr(), B, H, N, d, blk, _stream(stream)), "solattn_pool")
+    return out
+
+
+def solattn_forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, Bq: int, Bk: int, tau: float,
+                    mode="keep_correct", out: torch.Tensor | None = None,
+                    kept_per_head: torch.Tensor | None = None, keep_mask: bool | torch.Tensor = False,
+                    workspace: torch.Tensor | None = None, stream=None, events=None):
+    """Run the Sol-Attn forward operator on bf16 [B, H, N, d] CUDA tensors.
+
+    ``events``: optional pair of ``torch.cuda.Event(enable_timing=True)`` recorded
+    around the attention kernel (solattn_forward_events).
+
+    Returns (out bf16 [B, H, N, d], kept_per_head int64 [B, H], keep_mask uint32
+    [B, H, nQB, ceil(nKB/32)] or None). Asynchronous on ``stream``; device-side
+    errors are reported by :func:`solattn_get_status` on the workspace.
+    """
+    B, H, N, d = _bhnd(q)
+    for t in (q, k, v):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous() or tuple(t.shape) != (B, H, N, d):
+            raise ValueError("q, k, v must be contiguous bf16 CUDA tensors of one shape")
+    dev = q.device
+    if out is None:
+        out = torch.empty_like(q)
+    if kept_per_head is None:
+        kept_per_head = torch.empty((B, H), dtype=torch.int64, device=dev)
+    mask = None
+    if isinstance(keep_mask, torch.Tensor):
+        mask = keep_mask
+    elif keep_mask:
+        nq, nk = -(-N // Bq), -(-N // Bk)
+        mask = torch.empty((B, H, nq, -(-nk // 32)), dtype=torch.int32, device=dev)
+    if workspace is None:
+        workspace = alloc_workspace(B, H, N, d, Bq, Bk, dev)
+    stats = _Stats(kept_per_head.data_ptr(), mask.data_ptr() if mask is not None else None)
+    args = (q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, H, N, d, Bq, Bk,
+            ctypes.c_float(float(tau)), _mode(mode), ctypes.byref(stats), workspace.data_ptr(),
+            workspace.numel(), _stream(stream))
+    if events is None:
+        rc = _lib.solattn_forward(*args)
+    else:
+        rc = _lib.solattn_forward_events(*args, ctypes.c_void_p(events[0].cuda_event),
+                                         ctypes.c_void_p(events[1].cuda_event))
+    _check(rc, "solattn_forward")
+    return out, kept_per_head, mask
+
+
+def solattn_get_status(workspace: torch.Tensor, stream=None) -> int:
+    return int(_lib.solattn_get_status(workspace.data_ptr(), _stream(stream)))
+
+
+def solattn_forward_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, Bq: int, Bk: int, tau: float,
+                         mode="keep_correct", out: torch.Tensor | None = None,
+                         kept_per_head: torch.Tensor | None = None, scratch: torch.Tensor | None = None,
+                         stream=None):
+    """End-to-end call on HOST (ideally pinned) bf16 tensors: host->device copies,
+    the operator, and device->host copies of the output and per-head counts, all
+    inside the library call, which returns after the stream is synchronised."""
+    B, H, N, d = _bhnd(q)
+    for t in (q, k, v):
+        if t.dtype != torch.bfloat16 or t.is_cuda or not t.is_contiguous():
+            raise ValueError("q, k, v must be contiguous bf16 host tensors")
+    if out is None:
+        out = torch.empty_like(q, pin_memory=True)
+    if kept_per_head is None:
+        kept_per_head = torch.empty((B, H), dtype=torch.int64)
+    need = solattn_host_workspace_size(B, H, N, d, Bq, Bk)
+    if scratch is None:
+        scratch = torch.empty(need, dtype=torch.uint8, device="cuda")
+    rc = _lib.solattn_forward_host(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, H, N, d, Bq, Bk,
+                                   ctypes.c_float(float(tau)), _mode(mode), kept_per_head.data_ptr(),
+                                   scratch.data_ptr(), scratch.numel(), _stream(stream))
+    _check(rc, "solattn_forward_host")
+    return out, kept_per_head
+
+
+def solattn_watchdog_selftest(limit_ns: int = 2_000_000, stream=None) -> int:
+    """Run the device watchdog self-test; returns the status the kernel stored
+    (SOLATTN_ETIMEOUT when a wait that nobody completes is abandoned on time)."""
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    _check(_lib.solattn_watchdog_selftest(ws.data_ptr(), ws.numel(), int(limit_ns), _stream(stream)),
+           "solattn_watchdog_selftest")
+    return solattn_get_status(ws, stream)
+
+
+__all__ = [n for n in globals() if n.startswith("solattn_")] + ["SolAttnError", "MODES"]

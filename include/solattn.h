@@ -1,0 +1,175 @@
+/*
+ * solattn.h -- C ABI of libsolattn, a B200 (sm_100a) implementation of the
+ * Sol-Attn forward attention operator.
+ *
+ * Sol-Attn ("Sol-Attn: Accelerating Video Generation Inference via On-the-Fly
+ * Attention Sparsification", abstract and paperlayer summary §3 Methodology)
+ * runs one online-softmax pass over key/value blocks. For every query block it
+ * scores each key block with a proxy taken from the mean-pooled Q and K blocks,
+ * keeps the block for exact attention only if the proxy clears a threshold set
+ * relative to the running maximum, and folds every dropped block back in as one
+ * pseudo-key that carries the block's mean V ("approximate correction" by
+ * proxy-score reuse). The proxy map is never written to memory.
+ *
+ * Definitions used here (the pages leave these open; this library fixes them):
+ *   q_i, k_j, v_j  means of Q, K, V over the VALID rows of query block i /
+ *                  key block j (a ragged last block divides by its row count n_j)
+ *   s_ij           = q_i . k_j / sqrt(d)                          (block proxy)
+ *   visit order    query block i visits key blocks (j0 + t) mod nKB,
+ *                  t = 0..nKB-1, with j0 = min(floor(i*Bq/Bk), nKB-1)
+ *   threshold      M = max of the proxies visited so far (current included);
+ *                  the visited block is kept iff s_ij >= M - tau
+ *   output row r   keep_correct: [sum_kept sum_c e^{s_rc} v_c + sum_dropped n_j e^{s_ij} v_j]
+ *                               / [sum_kept sum_c e^{s_rc} + sum_dropped n_j e^{s_ij}]
+ *                  keep_drop:    the same without the dropped terms
+ *                  dense:        every block kept (plain softmax attention)
+ *   with s_rc = q_r . k_c / sqrt(d).
+ *
+ * Data layout: q, k, v and out are contiguous row-major bf16 [B][H][N][d]
+ * (token index n = (t*Y + y)*X + x for a (t, y, x) patch grid, t-major).
+ * Pooled buffers are contiguous fp32 [B][H][nB][d].
+ *
+ * Threading: every entry point that takes a stream enqueues work on that
+ * CUDA stream (cudaStream_t passed as void*, NULL = legacy default stream)
+ * and returns without waiting, except solattn_get_status and
+ * solattn_forward_host, which synchronise the stream.
+ *
+ * Ownership: the caller allocates and owns every buffer (inputs, output,
+ * statistics, workspace). The library keeps no allocation between calls.
+ */
+#ifndef SOLATTN_H
+#define SOLATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Routing / correction mode. */
+typedef enum {
+  SOLATTN_DENSE = 0,        /* every key block kept: plain softmax attention        */
+  SOLATTN_KEEP_DROP = 1,    /* dropped blocks discarded ("keep-or-drop")             */
+  SOLATTN_KEEP_CORRECT = 2  /* dropped blocks re-enter as proxy-weighted pseudo-keys */
+} solattn_mode;
+
+/* Status codes. Argument errors are returned before any device work is queued. */
+typedef enum {
+  SOLATTN_OK = 0,
+  SOLATTN_EINVAL = -1,       /* null pointer, misaligned pointer, N/B/H < 1, bad mode, tau < 0 or NaN */
+  SOLATTN_EUNSUPPORTED = -2, /* d not in {64,128}, Bq/Bk not in {64,128}, too many blocks, no sm_100 device */
+  SOLATTN_ECUDA = -3,        /* a CUDA runtime or driver call failed                          */
+  SOLATTN_ETIMEOUT = -4,     /* a device-side wait ran past its limit (reported by get_status) */
+  SOLATTN_EWORKSPACE = -5    /* workspace pointer null/misaligned or smaller than required     */
+} solattn_status;
+
+/* Per-call statistics (device pointers). */
+typedef struct {
+  /* [B*H] int64: sum over query blocks i of |K_i| (kept key blocks) for each
+   * (b, h). Required. Overwritten by every solattn_forward call; in dense mode
+   * it is nQB*nKB. */
+  int64_t *kept_per_head;
+  /* Optional (NULL to skip): [B*H][nQB][ceil(nKB/32)] uint32 keep bit-mask,
+   * bit (j & 31) of word (j >> 5) set iff query block i keeps key block j.
+   * Overwritten for every valid query block. For tests; off the timed path. */
+  uint32_t *keep_mask;
+} solattn_stats;
+
+/* Largest number of key blocks per head (nKB = ceil(N/Bk)) a call accepts. */
+#define SOLATTN_MAX_KEY_BLOCKS 1024
+
+/*
+ * Bytes of device workspace solattn_forward needs for this shape: a small
+ * header (work counter, device status word) plus the pooled q, k, v blocks in
+ * fp32. Returns 0 for an unsupported or invalid shape.
+ */
+size_t solattn_workspace_size(int B, int H, int N, int d, int Bq, int Bk);
+
+/*
+ * Mean-pool one bf16 tensor x [B][H][N][d] over blocks of `blk` rows into
+ * xbar [B][H][ceil(N/blk)][d] fp32 (ragged last block: mean over its valid
+ * rows). Step "mean pooling of each query and key block" (paperlayer summary
+ * §2 Preliminaries; §3 Methodology, "pooled keys and summed values").
+ * x must be 16-byte aligned, xbar 16-byte aligned. blk in {64,128}, d in {64,128}.
+ * Returns SOLATTN_OK or an error code; asynchronous on `stream`.
+ */
+int solattn_pool(const void *x, float *xbar, int B, int H, int N, int d, int blk,
+                 void *stream);
+
+/*
+ * The Sol-Attn forward operator (one fused pass per query tile: routing,
+ * exact attention on kept blocks, correction for dropped blocks; abstract and
+ * paperlayer summary §3 Methodology, "Unified execution").
+ *
+ *   q, k, v    device, bf16 [B][H][N][d], 16-byte aligned
+ *   out        device, bf16 [B][H][N][d], 16-byte aligned (written)
+ *   B, H, N    batch, heads, tokens (>= 1); nKB = ceil(N/Bk) <= SOLATTN_MAX_KEY_BLOCKS
+ *   d          head dim, 64 or 128
+ *   Bq, Bk     query / key block sizes, each 64 or 128
+ *   tau        threshold offset in logit units, >= 0; +INFINITY keeps every block;
+ *              ignored in dense mode
+ *   mode       a solattn_mode
+ *   stats      required; stats->kept_per_head device [B*H] int64
+ *   workspace  device, 256-byte aligned, >= solattn_workspace_size(...) bytes;
+ *              must not be used by another call that runs at the same time
+ *   stream     cudaStream_t (as void*)
+ *
+ * Returns SOLATTN_OK once the work is queued (errors inside the kernels are
+ * reported by solattn_get_status), or an error code with nothing queued.
+ */
+int solattn_forward(const void *q, const void *k, const void *v, void *out,
+                    int B, int H, int N, int d, int Bq, int Bk, float tau, int mode,
+                    const solattn_stats *stats, void *workspace, size_t ws_bytes,
+                    void *stream);
+
+/*
+ * solattn_forward plus two CUDA events (cudaEvent_t as void*, either may be NULL)
+ * recorded on `stream` immediately before and after the attention kernel, so a
+ * caller can time that kernel alone inside a timed region. Same arguments,
+ * results and errors as solattn_forward.
+ */
+int solattn_forward_events(const void *q, const void *k, const void *v, void *out,
+                           int B, int H, int N, int d, int Bq, int Bk, float tau, int mode,
+                           const solattn_stats *stats, void *workspace, size_t ws_bytes,
+                           void *stream, void *ev_attn_begin, void *ev_attn_end);
+
+/*
+ * Synchronise `stream` and read the device status word of `workspace`
+ * (SOLATTN_OK, or SOLATTN_ETIMEOUT if a bounded device-side wait gave up).
+ */
+int solattn_get_status(const void *workspace, void *stream);
+
+/* Bytes of device scratch solattn_forward_host needs (device copies of q, k,
+ * v, out, the per-head counts and the forward workspace). 0 if invalid. */
+size_t solattn_host_workspace_size(int B, int H, int N, int d, int Bq, int Bk);
+
+/*
+ * End-to-end call on HOST buffers: copies q, k, v (bf16 [B][H][N][d], host,
+ * ideally pinned) to the device scratch, runs solattn_forward, copies the bf16
+ * output to `out` and the per-head kept counts to `kept_per_head` (host int64
+ * [B*H], may be NULL), then synchronises `stream` and returns the device status.
+ * dev_scratch: device, 256-byte aligned, >= solattn_host_workspace_size(...).
+ */
+int solattn_forward_host(const void *q, const void *k, const void *v, void *out,
+                         int B, int H, int N, int d, int Bq, int Bk, float tau, int mode,
+                         int64_t *kept_per_head, void *dev_scratch, size_t scratch_bytes,
+                         void *stream);
+
+/*
+ * Self-test of the device watchdog: launches one block that waits on a
+ * barrier nobody completes, with a limit of `limit_ns` nanoseconds, and
+ * stores the resulting status (SOLATTN_ETIMEOUT when the watchdog works) in
+ * the workspace status word. Read it with solattn_get_status.
+ */
+int solattn_watchdog_selftest(void *workspace, size_t ws_bytes, uint64_t limit_ns,
+                              void *stream);
+
+/* Static description of a status code. */
+const char *solattn_strerror(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SOLATTN_H */

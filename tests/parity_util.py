@@ -1,0 +1,73 @@
+"""Shared helpers of the GPU parity tests: run the CUDA path through the C ABI and
+compare it with the fp64 oracle on the same bf16 inputs."""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import torch
+
+import oracle.solattn_ref as ref
+
+# Tolerances (bf16 inputs, fp32 accumulation): max-abs error of the bf16 output and the
+# L1-relative error sum|o - o_ref| / sum|o_ref| over every checked element; kept-set
+# differences are allowed only where the oracle's proxy is within NEAR of the threshold.
+MAX_ABS = 1e-2
+MEAN_REL = 2e-3
+NEAR = 1e-3
+
+
+def unpack_mask(mask: torch.Tensor, nKB: int) -> np.ndarray:
+    m = mask.cpu().contiguous().numpy().view(np.uint32)
+    bits = np.unpackbits(m.view(np.uint8), bitorder="little").reshape(m.shape[:-1] + (-1,))
+    return bits[..., :nKB].astype(bool)
+
+
+def run_gpu(q, k, v, Bq, Bk, tau, mode):
+    from block_sparse_online_b200 import solattn
+    dev = torch.device("cuda:0")
+    qd, kd, vd = (t.to(dev).contiguous() for t in (q, k, v))
+    ws = solattn.alloc_workspace(*qd.shape, Bq, Bk, dev)
+    out, kept, mask = solattn.solattn_forward(qd, kd, vd, Bq, Bk, tau, mode, keep_mask=True, workspace=ws)
+    st = solattn.solattn_get_status(ws)
+    assert st == 0, f"device status {st}"
+    torch.cuda.synchronize()
+    return out.cpu(), kept.cpu(), mask
+
+
+def check_case(q, k, v, Bq, Bk, tau, mode, qblocks=None, label=""):
+    """Run one case on the GPU and compare keep sets, counts and outputs with the oracle.
+    Returns a dict of the measured errors."""
+    B, H, N, d = q.shape
+    nQB, nKB = -(-N // Bq), -(-N // Bk)
+    out, kept, mask = run_gpu(q, k, v, Bq, Bk, tau, mode)
+    gpu_keep = unpack_mask(mask, nKB)
+    ref_keep, margin, _ = ref.keep_sets(q, k, Bq, Bk, tau, mode)
+    diff = gpu_keep != ref_keep
+    flips = int(diff.sum())
+    if flips:
+        worst = float(np.abs(margin[diff]).max())
+        assert worst < NEAR, f"{label}: keep set differs away from the threshold (|margin| {worst})"
+    # per-head kept counts equal the GPU's own mask popcounts, and the oracle's where no flip
+    np.testing.assert_array_equal(kept.numpy(), gpu_keep.sum(axis=(-1, -2)))
+    if not flips:
+        np.testing.assert_array_equal(kept.numpy(), ref.kept_per_head(ref_keep))
+    want, _ = ref.forward(q, k, v, Bq, Bk, tau, mode, keep=gpu_keep, qblocks=qblocks)
+    got = out.to(torch.float64).numpy()
+    sel = ~np.isnan(want[..., 0])
+    w, g = want[sel], got[sel]
+    assert np.isfinite(g).all(), f"{label}: non-finite output"
+    max_abs = float(np.abs(g - w).max())
+    mean_rel = float(np.abs(g - w).sum() / np.abs(w).sum())
+    assert max_abs <= MAX_ABS, f"{label}: max abs error {max_abs}"
+    assert mean_rel <= MEAN_REL, f"{label}: mean relative error {mean_rel}"
+    return {"flips": flips, "max_abs": max_abs, "mean_rel": mean_rel,
+            "keep_ratio": float(gpu_keep.mean()), "rows": int(sel.sum())}
+
+
+def sampled_blocks(B, H, N, Bq, Bk, per_head, seed=0):
+    nQB, nKB = -(-N // Bq), -(-N // Bk)
+    return ref.sample_qblocks(B, H, nQB, Bq, Bk, nKB, per_head=per_head, seed=seed)
+
+
+__all__ = ["check_case", "run_gpu", "unpack_mask", "sampled_blocks", "MAX_ABS", "MEAN_REL", "NEAR", "math"]

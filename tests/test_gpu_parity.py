@@ -1,0 +1,158 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle.
+
+Kept-block sets must match bit for bit except where the oracle's proxy lies
+within 1e-3 of the threshold; outputs must stay within max-abs 1e-2 and
+L1-relative 2e-3 (bf16 inputs, fp32 accumulation), computed on the GPU's own
+keep set. Small cases are checked on every row; the full-size configurations
+on a seeded sample of query blocks per head (block 0, the middle one and the
+ragged last one always included).
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle.solattn_ref as ref
+from block_sparse_online_b200 import synth
+from tests.parity_util import check_case, run_gpu, sampled_blocks, unpack_mask
+
+pytestmark = pytest.mark.gpu
+INF = math.inf
+MODES = ("dense", "keep_drop", "keep_correct")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+
+
+# ------------------------------------------------------------ small shapes, all rows
+
+@pytest.mark.parametrize("mode", MODES)
+@pytest.mark.parametrize("tau", [2.0, 4.0, INF])
+def test_tiny_config(mode, tau):
+    q, k, v = synth.make_inputs("tiny")
+    check_case(q, k, v, 64, 64, tau, mode, label=f"tiny {mode} {tau}")
+
+
+SHAPES = [
+    # (B, H, N, d, Bq, Bk): ragged tails, Bq != Bk, single partial tile, odd tile counts
+    (1, 1, 1000, 64, 64, 64),
+    (1, 2, 777, 128, 128, 64),
+    (2, 1, 777, 128, 64, 128),
+    (1, 1, 50, 64, 64, 64),
+    (1, 1, 129, 128, 128, 128),
+    (1, 3, 640, 128, 128, 128),
+    (2, 2, 1300, 64, 128, 128),
+    (1, 1, 2000, 128, 64, 64),
+]
+
+
+@pytest.mark.parametrize("shape", SHAPES, ids=[str(s) for s in SHAPES])
+@pytest.mark.parametrize("mode", MODES)
+def test_shapes(shape, mode):
+    B, H, N, d, Bq, Bk = shape
+    cfg = synth.Config("adhoc", B=B, H=H, d=d, grid=(1, 1, N), Bq=Bq, Bk=Bk, taus=(), seed=11 + N)
+    q, k, v = synth.make_inputs(cfg)
+    for tau in (0.0, 1.5, 3.0):
+        check_case(q, k, v, Bq, Bk, tau, mode, label=f"{shape} {mode} {tau}")
+
+
+def test_random_inputs_extreme_logits():
+    # Large logits (std ~ 8) stress the lazy rescaling of the running max.
+    q, k, v = synth.make_random(1, 2, 900, 128, seed=3, scale=2.2)
+    for mode in MODES:
+        check_case(q, k, v, 128, 128, 2.0, mode, label=f"extreme {mode}")
+
+
+def test_constant_blocks_correction_exact_on_gpu():
+    """Constant Q rows per query block and K rows per key block: keep_correct equals dense."""
+    g = torch.Generator().manual_seed(5)
+    N, d, blk = 1000, 128, 128
+    nb = -(-N // blk)
+    qb = torch.randn(nb, d, generator=g) * 0.6
+    kb = torch.randn(nb, d, generator=g) * 0.6
+    q = qb.repeat_interleave(blk, 0)[:N].to(torch.bfloat16)[None, None].contiguous()
+    k = kb.repeat_interleave(blk, 0)[:N].to(torch.bfloat16)[None, None].contiguous()
+    v = torch.randn(1, 1, N, d, generator=g).to(torch.bfloat16)
+    dense, _, _ = run_gpu(q, k, v, blk, blk, 0.0, "dense")
+    for tau in (0.0, 1.0):
+        out, kept, mask = run_gpu(q, k, v, blk, blk, tau, "keep_correct")
+        assert unpack_mask(mask, nb).mean() < 1.0
+        err = (out.float() - dense.float()).abs().max().item()
+        assert err <= 1e-2, err
+
+
+def test_tau_inf_equals_dense_bitwise():
+    q, k, v = synth.make_inputs("tiny")
+    d_out, d_kept, _ = run_gpu(q, k, v, 64, 64, 0.0, "dense")
+    for mode in ("keep_drop", "keep_correct"):
+        out, kept, _ = run_gpu(q, k, v, 64, 64, INF, mode)
+        assert torch.equal(out, d_out)
+        assert torch.equal(kept, d_kept)
+
+
+def test_deterministic():
+    cfg = synth.small_config(N=3000, d=128, Bq=128, Bk=128, H=3)
+    q, k, v = synth.make_inputs(cfg)
+    a = run_gpu(q, k, v, 128, 128, 3.0, "keep_correct")
+    b = run_gpu(q, k, v, 128, 128, 3.0, "keep_correct")
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1]) and torch.equal(a[2].cpu(), b[2].cpu())
+
+
+def test_pool_matches_oracle():
+    from block_sparse_online_b200 import solattn
+    q, _, _ = synth.make_random(2, 3, 1111, 128, seed=9)
+    for blk in (64, 128):
+        got = solattn.solattn_pool(q.cuda(), blk).cpu().double().numpy()
+        want = ref.pool(q, blk)
+        np.testing.assert_allclose(got, want, rtol=1e-5, atol=1e-6)
+
+
+def test_watchdog_reports_timeout():
+    from block_sparse_online_b200 import solattn
+    assert solattn.solattn_watchdog_selftest(limit_ns=2_000_000) == solattn.SOLATTN_ETIMEOUT
+
+
+def test_host_entry_point_matches_device_call():
+    from block_sparse_online_b200 import solattn
+    q, k, v = synth.make_inputs("tiny")
+    dev_out, dev_kept, _ = run_gpu(q, k, v, 64, 64, 2.0, "keep_correct")
+    qh, kh, vh = (t.pin_memory() for t in (q, k, v))
+    out, kept = solattn.solattn_forward_host(qh, kh, vh, 64, 64, 2.0, "keep_correct")
+    assert torch.equal(out, dev_out)
+    assert torch.equal(kept, dev_kept)
+
+
+# ------------------------------------------------------------ full-size configurations
+
+def _full(name, taus, modes, per_head):
+    cfg = synth.CONFIGS[name]
+    q, k, v = synth.make_inputs(cfg)
+    blocks = sampled_blocks(cfg.B, cfg.H, cfg.N, cfg.Bq, cfg.Bk, per_head, seed=cfg.seed)
+    stats = {}
+    for mode in modes:
+        for tau in (taus if mode != "dense" else (0.0,)):
+            stats[(mode, tau)] = check_case(q, k, v, cfg.Bq, cfg.Bk, tau, mode, qblocks=blocks,
+                                            label=f"{name} {mode} {tau}")
+    return stats
+
+
+def test_image_config():
+    _full("image", (2.0, 4.0, 6.0, INF), MODES, per_head=2)
+
+
+def test_video480_config():
+    _full("video480", (2.0, 3.0, 4.0, 6.0, INF), MODES, per_head=6)
+
+
+@pytest.mark.slow
+def test_video720_config():
+    _full("video720", (3.0, 4.0, 6.0), MODES, per_head=3)
+
+
+@pytest.mark.slow
+def test_long_config():
+    _full("long", (3.0, 4.0, 6.0, INF), MODES, per_head=2)

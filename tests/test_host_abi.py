@@ -1,0 +1,109 @@
+"""Host-side tests of libsolattn (no GPU needed): the library loads, exports every
+symbol include/solattn.h declares, sizes workspaces, and rejects bad arguments
+before queueing any device work."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+from block_sparse_online_b200 import solattn
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "solattn.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(solattn_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for must in ("solattn_pool", "solattn_forward", "solattn_get_status", "solattn_workspace_size",
+                 "solattn_strerror"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(solattn.library_path())
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    assert set(declared_functions()) == set(solattn.EXPORTS)
+
+
+def test_strerror():
+    assert solattn.strerror(0) == "ok"
+    assert "timed out" in solattn.strerror(solattn.SOLATTN_ETIMEOUT)
+    assert solattn.strerror(12345) == "unknown status"
+
+
+def test_workspace_sizes():
+    ws = solattn.solattn_workspace_size
+    assert ws(1, 12, 32760, 128, 128, 128) > 12 * 256 * 128 * 4 * 3
+    assert ws(1, 1, 100, 96, 128, 128) == 0          # d unsupported
+    assert ws(1, 1, 100, 128, 32, 128) == 0          # block size unsupported
+    assert ws(1, 1, 0, 128, 128, 128) == 0           # empty
+    assert ws(1, 1, 1024 * 128, 128, 128, 128) > 0   # at the key-block limit
+    assert ws(1, 1, 1024 * 128 + 1, 128, 128, 128) == 0
+    assert solattn.solattn_host_workspace_size(1, 2, 1000, 64, 64, 64) > 4 * 2 * 1000 * 64 * 2
+
+
+def _call(**kw):
+    """solattn_forward with placeholder pointers. Every case passed here carries an
+    invalid argument, so the call must return before touching the device. The test
+    only runs where no GPU is visible, so a missed check cannot reach a kernel."""
+    a = dict(q=4096, k=4096, v=4096, out=4096, B=1, H=1, N=256, d=128, Bq=128, Bk=128, tau=2.0, mode=2,
+             kept=4096, mask=None, ws=4096, ws_bytes=1 << 30)
+    a.update(kw)
+    st = solattn._Stats(a["kept"], a["mask"])
+    return solattn._lib.solattn_forward(a["q"], a["k"], a["v"], a["out"], a["B"], a["H"], a["N"], a["d"], a["Bq"],
+                                        a["Bk"], ctypes.c_float(a["tau"]), a["mode"], ctypes.byref(st), a["ws"],
+                                        a["ws_bytes"], None)
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="placeholder pointers are used only without a GPU")
+@pytest.mark.parametrize("kw,want", [
+    (dict(q=None), solattn.SOLATTN_EINVAL),
+    (dict(out=None), solattn.SOLATTN_EINVAL),
+    (dict(kept=None), solattn.SOLATTN_EINVAL),
+    (dict(N=0), solattn.SOLATTN_EINVAL),
+    (dict(B=0), solattn.SOLATTN_EINVAL),
+    (dict(d=96), solattn.SOLATTN_EUNSUPPORTED),
+    (dict(Bq=32), solattn.SOLATTN_EUNSUPPORTED),
+    (dict(Bk=256), solattn.SOLATTN_EUNSUPPORTED),
+    (dict(N=200000, Bk=128), solattn.SOLATTN_EUNSUPPORTED),
+    (dict(mode=3), solattn.SOLATTN_EINVAL),
+    (dict(mode=-1), solattn.SOLATTN_EINVAL),
+    (dict(tau=-0.5), solattn.SOLATTN_EINVAL),
+    (dict(tau=float("nan")), solattn.SOLATTN_EINVAL),
+    (dict(q=4100), solattn.SOLATTN_EINVAL),          # not 16-byte aligned
+    (dict(kept=4100), solattn.SOLATTN_EINVAL),       # not 8-byte aligned
+    (dict(ws=None), solattn.SOLATTN_EWORKSPACE),
+    (dict(ws=4096 + 64), solattn.SOLATTN_EWORKSPACE),  # not 256-byte aligned
+    (dict(ws_bytes=100), solattn.SOLATTN_EWORKSPACE),
+])
+def test_forward_rejects_bad_arguments(kw, want):
+    assert _call(**kw) == want
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="placeholder pointers are used only without a GPU")
+def test_forward_without_device_reports_cuda_error():
+    # Valid arguments on a machine without a GPU: the device query fails cleanly.
+    assert _call() in (solattn.SOLATTN_ECUDA, solattn.SOLATTN_EUNSUPPORTED)
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="placeholder pointers are used only without a GPU")
+def test_pool_rejects_bad_arguments():
+    f = solattn._lib.solattn_pool
+    assert f(None, 4096, 1, 1, 128, 128, 128, None) == solattn.SOLATTN_EINVAL
+    assert f(4096, 4096, 1, 1, 128, 96, 128, None) == solattn.SOLATTN_EUNSUPPORTED
+    assert f(4104, 4096, 1, 1, 128, 128, 128, None) == solattn.SOLATTN_EINVAL
+
+
+def test_binding_rejects_cpu_tensors():
+    q = torch.zeros(1, 1, 64, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        solattn.solattn_forward(q, q, q, 64, 64, 1.0, "keep_drop")
