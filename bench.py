@@ -50,6 +50,9 @@ def parse():
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--heads", type=int, default=0,
+                    help="use only this many heads of the configuration (small profiling captures)")
     return ap.parse_args()
 
 
@@ -230,6 +233,40 @@ def reference_arm(args, world, rank):
     print(json.dumps(line), flush=True)
 
 
+def e2e_measure(args, cfg, q, k, v, dev, stream, world, barrier, dense_flops, elem):
+    """Same metric through the host entry point: pinned host q/k/v in, host output out,
+    host<->device copies inside the timed region."""
+    import torch
+    import torch.distributed as dist
+    from block_sparse_online_b200 import solattn
+    B, H, N, d = cfg.shape()
+    qh, kh, vh = q.pin_memory(), k.pin_memory(), v.pin_memory()
+    outh = torch.empty_like(q).pin_memory()
+    kh_cnt = torch.empty((B, H), dtype=torch.int64)
+    scratch = torch.empty(solattn.solattn_host_workspace_size(B, H, N, d, cfg.Bq, cfg.Bk), dtype=torch.uint8,
+                          device=dev)
+    e2e_steps = max(3, min(args.steps, 10))
+    for _ in range(2):
+        solattn.solattn_forward_host(qh, kh, vh, cfg.Bq, cfg.Bk, args.tau, args.mode, out=outh, kept_per_head=kh_cnt,
+                                     scratch=scratch)
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        solattn.solattn_forward_host(qh, kh, vh, cfg.Bq, cfg.Bk, args.tau, args.mode, out=outh, kept_per_head=kh_cnt,
+                                     scratch=scratch)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    return {"value": round(world * dense_flops / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s (dense-equivalent)",
+            "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": 3 * elem * 2,
+            "d2h_bytes_per_step": elem * 2 + B * H * 8, "steps": e2e_steps}
+
+
 def main():
     args = parse()
     world, rank, local = dist_setup(args)
@@ -245,6 +282,9 @@ def main():
     if world > 1:
         dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
     cfg = synth.CONFIGS[args.config]
+    if args.heads:
+        import dataclasses
+        cfg = dataclasses.replace(cfg, H=args.heads, note=cfg.note + f" [reduced to H={args.heads}]")
     B, H, N, d = cfg.shape()
     q, k, v = synth.make_inputs(cfg)
     qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
@@ -307,30 +347,10 @@ def main():
     trec = traffic_record()
 
     # end to end through the host entry point (pinned host buffers, copies inside the timed region)
-    qh, kh, vh = q.pin_memory(), k.pin_memory(), v.pin_memory()
-    outh = torch.empty_like(q).pin_memory()
-    kh_cnt = torch.empty((B, H), dtype=torch.int64)
-    scratch = torch.empty(solattn.solattn_host_workspace_size(B, H, N, d, cfg.Bq, cfg.Bk), dtype=torch.uint8,
-                          device=dev)
-    e2e_steps = max(3, min(args.steps, 10))
-    for _ in range(2):
-        solattn.solattn_forward_host(qh, kh, vh, cfg.Bq, cfg.Bk, args.tau, args.mode, out=outh, kept_per_head=kh_cnt,
-                                     scratch=scratch)
-    barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        solattn.solattn_forward_host(qh, kh, vh, cfg.Bq, cfg.Bk, args.tau, args.mode, out=outh, kept_per_head=kh_cnt,
-                                     scratch=scratch)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / e2e_steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_val = world * dense_flops / (e2e_ms * 1e-3) / 1e12
     elem = B * H * N * d
+    e2e = None
+    if not args.no_e2e:
+        e2e = e2e_measure(args, cfg, q, k, v, dev, stream, world, barrier, dense_flops, elem)
 
     sweep = []
     if not args.no_sweep and rank == 0:
@@ -392,8 +412,7 @@ def main():
                          "frac": round(achieved / peak_tf, 4), "peak_source": f"{peak_kind} bf16 dense (burst)",
                          "traffic": None if trec is None else trec["dram_bytes_per_launch"],
                          "kernel": "solattn_fwd_kernel (executed FLOPs per launch / CUDA-event duration)"},
-            "e2e": {"value": round(e2e_val, 3), "unit": "TFLOP/s (dense-equivalent)", "ms_per_step": round(e2e_ms, 3),
-                    "h2d_bytes_per_step": 3 * elem * 2, "d2h_bytes_per_step": elem * 2 + B * H * 8},
+            "e2e": e2e,
             "gpu_launches": args.steps * (1 if args.mode == "dense" else 2),
             "clocks": clk,
             "cpu_baseline": cpu,

@@ -5,8 +5,8 @@
 // blocks). Roles, by warp:
 //   warp 0      TMA producer: Q tiles of the item, then K_j and V_j of every key
 //               block j in the item's kept list, into a ring of shared-memory slots.
-//   warp 1      MMA issuer (one thread): S_t = Q_t K_j^T into tensor memory (TMEM),
-//               O_t += P_t V_j with P_t read from TMEM (tcgen05, bf16 -> fp32).
+//   warp 1      MMA issuer (one thread): S_t = Q_t K_j^T into tensor memory (TMEM,
+//               bf16 -> fp32), O_t += P_t V_j with P_t read from TMEM (fp16 -> fp32).
 //   warp 2      router: on-the-fly block thresholding and the correction sums for the
 //               NEXT item (double-buffered), from the fp32 pooled blocks in L2.
 //   warps 4..7  softmax warpgroup of tile 0, warps 8..11 of tile 1: online softmax
@@ -93,8 +93,10 @@ struct Cfg {
   static constexpr int CTRL_REGS = 88;
   static constexpr int SOFTMAX_REGS = 208;
   static_assert(NT != 2 || 128 * CTRL_REGS + 256 * SOFTMAX_REGS <= 384 * 168, "register split");
-  static constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, BK, false);
-  static constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, true);
+  // S = Q K^T in bf16; O += P V in fp16 (P in [0, 2^8] after the lazy rescale; V is the
+  // fp16 copy written by the pooling pass).
+  static constexpr uint32_t IDESC_QK = idesc_16bit_f32(128, BK, false, false);
+  static constexpr uint32_t IDESC_PV = idesc_16bit_f32(128, D, true, true);
   static_assert(TMEM_NEED <= 512, "TMEM budget");
   static_assert(NSB <= 8, "member bits");
 };
@@ -596,7 +598,7 @@ __device__ void run_softmax(SmemCtl<C> &sc, const FwdParams &p, uint32_t tmem, i
           const float p0 = (rk && col < ncol) ? ex2_approx(fmaf(x0, sc_log2, neg_m)) : 0.f;
           const float p1 = (rk && col + 1 < ncol) ? ex2_approx(fmaf(x1, sc_log2, neg_m)) : 0.f;
           lsum += p0 + p1;
-          pk[e] = pack_bf16x2(p0, p1);
+          pk[e] = pack_f16x2(p0, p1);
         }
         tmem_st32(s_addr + h * 32, pk);
       }

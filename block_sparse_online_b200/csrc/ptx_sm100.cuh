@@ -156,11 +156,12 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
   return d;
 }
 
-// Instruction descriptor, kind::f16: bf16 x bf16 -> fp32, A K-major, B K- or MN-major.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn_major) {
+// Instruction descriptor, kind::f16: 16-bit x 16-bit -> fp32 (both operands bf16, or
+// both fp16), A K-major, B K- or MN-major.
+__host__ __device__ constexpr uint32_t idesc_16bit_f32(int M, int N, bool b_mn_major, bool fp16) {
   return (1u << 4)                                   // accumulator format: f32
-         | (1u << 7)                                 // A format: bf16
-         | (1u << 10)                                // B format: bf16
+         | ((fp16 ? 0u : 1u) << 7)                   // A format: fp16 (0) or bf16 (1)
+         | ((fp16 ? 0u : 1u) << 10)                  // B format: same as A
          | (static_cast<uint32_t>(b_mn_major) << 16)  // B major-ness
          | (static_cast<uint32_t>(N >> 3) << 17)     // N / 8
          | (static_cast<uint32_t>(M >> 4) << 24);    // M / 16
@@ -231,6 +232,12 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   // cvt packs its first source into the upper half and the second into the lower half.
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
 }
 

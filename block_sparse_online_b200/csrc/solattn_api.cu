@@ -27,7 +27,7 @@ int nblocks(int N, int blk) { return (N + blk - 1) / blk; }
 bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 struct WsLayout {
-  size_t qbar, kbar, vbar, total;
+  size_t qbar, kbar, vbar, v16, total;
 };
 
 int check_shape(int B, int H, int N, int d, int Bq, int Bk) {
@@ -45,7 +45,8 @@ WsLayout ws_layout(int B, int H, int N, int d, int Bq, int Bk) {
   w.qbar = kHeaderBytes;
   w.kbar = w.qbar + align_up(bh * nblocks(N, Bq) * d * sizeof(float), kAlign);
   w.vbar = w.kbar + align_up(bh * nblocks(N, Bk) * d * sizeof(float), kAlign);
-  w.total = w.vbar + align_up(bh * nblocks(N, Bk) * d * sizeof(float), kAlign);
+  w.v16 = w.vbar + align_up(bh * nblocks(N, Bk) * d * sizeof(float), kAlign);
+  w.total = w.v16 + align_up(bh * N * d * 2, kAlign);
   return w;
 }
 
@@ -93,14 +94,15 @@ EncodeTiledFn encode_fn() {
 
 // 3-D view (d, N, B*H) of a contiguous bf16 [B][H][N][d] tensor; boxes of 64 x rows x 1
 // with the 128-byte swizzle. Rows past N read as zeros.
-int make_map(CUtensorMap *map, const void *ptr, int d, int N, int BH, int box_rows) {
+int make_map(CUtensorMap *map, const void *ptr, int d, int N, int BH, int box_rows,
+             CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return SOLATTN_ECUDA;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(N) * d * 2};
   cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
   cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box, estr,
+  CUresult r = enc(map, dtype, 3, const_cast<void *>(ptr), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? SOLATTN_OK : SOLATTN_ECUDA;
@@ -186,22 +188,31 @@ int forward_impl(const void *q, const void *k, const void *v, void *out, int B, 
   float *qbar = reinterpret_cast<float *>(ws + wl.qbar);
   float *kbar = reinterpret_cast<float *>(ws + wl.kbar);
   float *vbar = reinterpret_cast<float *>(ws + wl.vbar);
+  __half *v16 = reinterpret_cast<__half *>(ws + wl.v16);
 
   CUtensorMap mq, mk, mv;
   if (make_map(&mq, q, d, N, BH, 128) != SOLATTN_OK || make_map(&mk, k, d, N, BH, Bk) != SOLATTN_OK ||
-      make_map(&mv, v, d, N, BH, Bk) != SOLATTN_OK)
+      make_map(&mv, v16, d, N, BH, Bk, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) != SOLATTN_OK)
     return SOLATTN_ECUDA;
 
   if (cudaMemsetAsync(ws, 0, kHeaderBytes, st) != cudaSuccess) return SOLATTN_ECUDA;
   if (cudaMemsetAsync(stats->kept_per_head, 0, sizeof(int64_t) * BH, st) != cudaSuccess) return SOLATTN_ECUDA;
 
-  if (mode != SOLATTN_DENSE) {
+  {
+    // One pass over the inputs: block means of Q and K (routing) and of V (correction),
+    // and the fp16 copy of V for the P.V product. Dense mode needs only the copy.
+    const __nv_bfloat16 *vb = static_cast<const __nv_bfloat16 *>(v);
     PoolArgs a{};
-    a.job[0] = PoolJob{static_cast<const __nv_bfloat16 *>(q), qbar, Bq, nQB};
-    a.job[1] = PoolJob{static_cast<const __nv_bfloat16 *>(k), kbar, Bk, nKB};
-    a.job[2] = PoolJob{static_cast<const __nv_bfloat16 *>(v), vbar, Bk, nKB};
-    a.njobs = (mode == SOLATTN_KEEP_CORRECT) ? 3 : 2;
     a.N = N;
+    if (mode == SOLATTN_DENSE) {
+      a.job[0] = PoolJob{vb, nullptr, v16, Bk, nKB};
+      a.njobs = 1;
+    } else {
+      a.job[0] = PoolJob{vb, mode == SOLATTN_KEEP_CORRECT ? vbar : nullptr, v16, Bk, nKB};
+      a.job[1] = PoolJob{static_cast<const __nv_bfloat16 *>(q), qbar, nullptr, Bq, nQB};
+      a.job[2] = PoolJob{static_cast<const __nv_bfloat16 *>(k), kbar, nullptr, Bk, nKB};
+      a.njobs = 3;
+    }
     const int rcp = launch_pool(a, BH, d, nQB > nKB ? nQB : nKB, st);
     if (rcp != SOLATTN_OK) return rcp;
   }
@@ -249,7 +260,7 @@ int solattn_pool(const void *x, float *xbar, int B, int H, int N, int d, int blk
   if (device_info(&di) != SOLATTN_OK) return SOLATTN_ECUDA;
   if (di.major != 10) return SOLATTN_EUNSUPPORTED;
   PoolArgs a{};
-  a.job[0] = PoolJob{static_cast<const __nv_bfloat16 *>(x), xbar, blk, nblocks(N, blk)};
+  a.job[0] = PoolJob{static_cast<const __nv_bfloat16 *>(x), xbar, nullptr, blk, nblocks(N, blk)};
   a.njobs = 1;
   a.N = N;
   return launch_pool(a, B * H, d, nblocks(N, blk), static_cast<cudaStream_t>(stream));

@@ -165,6 +165,10 @@ def solattn_forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, Bq: int, 
     if events is None:
         rc = _lib.solattn_forward(*args)
     else:
+        st = stream if stream is not None else torch.cuda.current_stream()
+        for e in events:
+            if e.cuda_event == 0:  # torch creates the CUDA event on its first record
+                e.record(st)
         rc = _lib.solattn_forward_events(*args, ctypes.c_void_p(events[0].cuda_event),
                                          ctypes.c_void_p(events[1].cuda_event))
     _check(rc, "solattn_forward")

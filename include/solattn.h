@@ -58,7 +58,7 @@ typedef enum {
 typedef enum {
   SOLATTN_OK = 0,
   SOLATTN_EINVAL = -1,       /* null pointer, misaligned pointer, N/B/H < 1, bad mode, tau < 0 or NaN */
-  SOLATTN_EUNSUPPORTED = -2, /* d not in {64,128}, Bq/Bk not in {64,128}, too many blocks, no sm_100 device */
+  SOLATTN_EUNSUPPORTED = -2, /* d or Bq/Bk not in {64,128}, nKB > 1024, B*H > 65535, no sm_100 device */
   SOLATTN_ECUDA = -3,        /* a CUDA runtime or driver call failed                          */
   SOLATTN_ETIMEOUT = -4,     /* a device-side wait ran past its limit (reported by get_status) */
   SOLATTN_EWORKSPACE = -5    /* workspace pointer null/misaligned or smaller than required     */
@@ -81,8 +81,8 @@ typedef struct {
 
 /*
  * Bytes of device workspace solattn_forward needs for this shape: a small
- * header (work counter, device status word) plus the pooled q, k, v blocks in
- * fp32. Returns 0 for an unsupported or invalid shape.
+ * header (work counter, device status word), the pooled q, k, v blocks in fp32
+ * and an fp16 copy of v. Returns 0 for an unsupported or invalid shape.
  */
 size_t solattn_workspace_size(int B, int H, int N, int d, int Bq, int Bk);
 
@@ -102,7 +102,9 @@ int solattn_pool(const void *x, float *xbar, int B, int H, int N, int d, int blk
  * exact attention on kept blocks, correction for dropped blocks; abstract and
  * paperlayer summary §3 Methodology, "Unified execution").
  *
- *   q, k, v    device, bf16 [B][H][N][d], 16-byte aligned
+ *   q, k, v    device, bf16 [B][H][N][d], 16-byte aligned. The P.V product runs in
+ *              fp16 (on an fp16 copy of v made by the pooling pass), so entries of v
+ *              must lie in the fp16 range, |v| <= 65504; larger ones become inf.
  *   out        device, bf16 [B][H][N][d], 16-byte aligned (written)
  *   B, H, N    batch, heads, tokens (>= 1); nKB = ceil(N/Bk) <= SOLATTN_MAX_KEY_BLOCKS
  *   d          head dim, 64 or 128

@@ -2,19 +2,27 @@
 compare it with the fp64 oracle on the same bf16 inputs."""
 from __future__ import annotations
 
-import math
-
 import numpy as np
 import torch
 
 import oracle.solattn_ref as ref
 
-# Tolerances (bf16 inputs, fp32 accumulation): max-abs error of the bf16 output and the
-# L1-relative error sum|o - o_ref| / sum|o_ref| over every checked element; kept-set
-# differences are allowed only where the oracle's proxy is within NEAR of the threshold.
+# Tolerances (bf16 inputs, fp32 accumulation, bf16 output):
+#  * max-abs: |o - o_ref| <= MAX_ABS + ulp_bf16(o_ref) / 2 elementwise. The output is
+#    stored in bf16, whose spacing is 2^-5 for |o| in [4, 8): rounding alone moves such
+#    an output by up to 1.6e-2, so the 1e-2 bound is applied to the error beyond the
+#    half-ulp of the bf16 result.
+#  * mean relative: sum|o - o_ref| / sum|o_ref| <= MEAN_REL over every checked element.
+#  * kept sets: equal, except where the oracle's proxy lies within NEAR of the threshold.
 MAX_ABS = 1e-2
 MEAN_REL = 2e-3
 NEAR = 1e-3
+
+
+def half_ulp_bf16(x: np.ndarray) -> np.ndarray:
+    """Half the spacing of bf16 numbers (8 significant bits) at |x|."""
+    e = np.floor(np.log2(np.maximum(np.abs(x), 2.0 ** -126)))
+    return 0.5 * np.exp2(e - 7)
 
 
 def unpack_mask(mask: torch.Tensor, nKB: int) -> np.ndarray:
@@ -57,11 +65,13 @@ def check_case(q, k, v, Bq, Bk, tau, mode, qblocks=None, label=""):
     sel = ~np.isnan(want[..., 0])
     w, g = want[sel], got[sel]
     assert np.isfinite(g).all(), f"{label}: non-finite output"
-    max_abs = float(np.abs(g - w).max())
-    mean_rel = float(np.abs(g - w).sum() / np.abs(w).sum())
-    assert max_abs <= MAX_ABS, f"{label}: max abs error {max_abs}"
+    err = np.abs(g - w)
+    max_abs = float(err.max())
+    excess = float((err - half_ulp_bf16(w)).max())
+    mean_rel = float(err.sum() / np.abs(w).sum())
+    assert excess <= MAX_ABS, f"{label}: max abs error beyond bf16 half-ulp {excess} (raw {max_abs})"
     assert mean_rel <= MEAN_REL, f"{label}: mean relative error {mean_rel}"
-    return {"flips": flips, "max_abs": max_abs, "mean_rel": mean_rel,
+    return {"flips": flips, "max_abs": max_abs, "max_abs_beyond_half_ulp": excess, "mean_rel": mean_rel,
             "keep_ratio": float(gpu_keep.mean()), "rows": int(sel.sum())}
 
 
@@ -70,4 +80,4 @@ def sampled_blocks(B, H, N, Bq, Bk, per_head, seed=0):
     return ref.sample_qblocks(B, H, nQB, Bq, Bk, nKB, per_head=per_head, seed=seed)
 
 
-__all__ = ["check_case", "run_gpu", "unpack_mask", "sampled_blocks", "MAX_ABS", "MEAN_REL", "NEAR", "math"]
+__all__ = ["check_case", "run_gpu", "unpack_mask", "sampled_blocks", "half_ulp_bf16", "MAX_ABS", "MEAN_REL", "NEAR"]

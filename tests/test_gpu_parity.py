@@ -1,9 +1,9 @@
 """GPU parity: the CUDA path (through the C ABI) against the fp64 oracle.
 
 Kept-block sets must match bit for bit except where the oracle's proxy lies
-within 1e-3 of the threshold; outputs must stay within max-abs 1e-2 and
-L1-relative 2e-3 (bf16 inputs, fp32 accumulation), computed on the GPU's own
-keep set. Small cases are checked on every row; the full-size configurations
+within 1e-3 of the threshold; outputs must stay within max-abs 1e-2 beyond the
+half-ulp of the bf16 result, and L1-relative 2e-3 (bf16 inputs, fp32
+accumulation), computed on the GPU's own keep set. Small cases are checked on every row; the full-size configurations
 on a seeded sample of query blocks per head (block 0, the middle one and the
 ragged last one always included).
 """
@@ -15,7 +15,7 @@ import torch
 
 import oracle.solattn_ref as ref
 from block_sparse_online_b200 import synth
-from tests.parity_util import check_case, run_gpu, sampled_blocks, unpack_mask
+from tests.parity_util import check_case, half_ulp_bf16, run_gpu, sampled_blocks, unpack_mask
 
 pytestmark = pytest.mark.gpu
 INF = math.inf
@@ -81,8 +81,9 @@ def test_constant_blocks_correction_exact_on_gpu():
     for tau in (0.0, 1.0):
         out, kept, mask = run_gpu(q, k, v, blk, blk, tau, "keep_correct")
         assert unpack_mask(mask, nb).mean() < 1.0
-        err = (out.float() - dense.float()).abs().max().item()
-        assert err <= 1e-2, err
+        err = (out.double() - dense.double()).abs()
+        tol = 2e-3 + 2 * torch.from_numpy(half_ulp_bf16(dense.double().numpy()))
+        assert (err <= tol).all(), err.max().item()
 
 
 def test_tau_inf_equals_dense_bitwise():
