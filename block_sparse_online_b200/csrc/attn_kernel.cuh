@@ -33,7 +33,10 @@
 
 #include <cstdint>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <math_constants.h>
+
+#include <type_traits>
 
 #include "ptx_sm100.cuh"
 
@@ -90,8 +93,8 @@ struct Cfg {
   // Register split: the control warpgroup hands registers to the softmax warpgroups,
   // which hold a whole S row. The sum stays within the registers the block is
   // launched with (384 threads x 168).
-  static constexpr int CTRL_REGS = 88;
-  static constexpr int SOFTMAX_REGS = 208;
+  static constexpr int CTRL_REGS = 120;
+  static constexpr int SOFTMAX_REGS = 192;
   static_assert(NT != 2 || 128 * CTRL_REGS + 256 * SOFTMAX_REGS <= 384 * 168, "register split");
   // S = Q K^T in bf16; O += P V in fp16 (P in [0, 2^8] after the lazy rescale; V is the
   // fp16 copy written by the pooling pass).
@@ -117,7 +120,6 @@ template <class C>
 struct SmemCtl {
   RouteSlot<C> route[2];
   uint32_t mask[C::NSB][kMaskWords];  // router scratch: keep bits per query block
-  float qrow[C::D];                    // router scratch: pooled query block
   uint64_t full[C::NSLOT];
   uint64_t empty[C::NSLOT];
   uint64_t q_full, q_empty;
@@ -143,20 +145,80 @@ __device__ __forceinline__ float u2f(uint32_t x) { return __uint_as_float(x); }
 
 // ------------------------------------------------------------------ router
 
+// Warp transpose-sum: every lane holds 32 partial values v[0..31]; on return lane l
+// holds the sum over the 32 lanes of v[l]. A butterfly of 31 shuffles (16 + 8 + 4 + 2
+// + 1): at each stage a lane keeps the half of its values whose index bit matches its
+// own lane bit and adds the partner's copy of that half.
+__device__ __forceinline__ float warp_transpose_sum32(float (&v)[32], int lane) {
+#pragma unroll
+  for (int w = 16; w >= 1; w >>= 1) {
+    const bool hi = (lane & w) != 0;
+#pragma unroll
+    for (int i = 0; i < w; ++i) {
+      const float keep = hi ? v[i + w] : v[i];
+      const float send = hi ? v[i] : v[i + w];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, w);
+    }
+  }
+  return v[0];
+}
+
+template <int VPL>
+struct VecOf;
+template <>
+struct VecOf<4> {
+  using T = float4;
+  static __device__ __forceinline__ float dot(const float (&a)[4], const float4 &b) {
+    return fmaf(a[3], b.w, fmaf(a[2], b.z, fmaf(a[1], b.y, a[0] * b.x)));
+  }
+  static __device__ __forceinline__ void axpy(float (&acc)[4], float w, const float4 &b) {
+    acc[0] = fmaf(w, b.x, acc[0]);
+    acc[1] = fmaf(w, b.y, acc[1]);
+    acc[2] = fmaf(w, b.z, acc[2]);
+    acc[3] = fmaf(w, b.w, acc[3]);
+  }
+  static __device__ __forceinline__ float4 zero() { return make_float4(0.f, 0.f, 0.f, 0.f); }
+};
+template <>
+struct VecOf<2> {
+  using T = float2;
+  static __device__ __forceinline__ float dot(const float (&a)[2], const float2 &b) {
+    return fmaf(a[1], b.y, a[0] * b.x);
+  }
+  static __device__ __forceinline__ void axpy(float (&acc)[2], float w, const float2 &b) {
+    acc[0] = fmaf(w, b.x, acc[0]);
+    acc[1] = fmaf(w, b.y, acc[1]);
+  }
+  static __device__ __forceinline__ float2 zero() { return make_float2(0.f, 0.f); }
+};
+
+// Route one query block: visit its key blocks in order, keep those whose proxy clears
+// the running maximum minus tau, and (keep_correct) fold every dropped block into the
+// correction sums. Lane-per-dimension layout: each pooled row is one coalesced
+// 128/256-byte load across the warp, loads are issued 8 rows at a time, and the 32
+// per-block dot products of a chunk are finished with one transpose-sum.
 template <class C>
 __device__ __forceinline__ void route_query_block(SmemCtl<C> &sc, RouteSlot<C> &rs, const FwdParams &p,
                                                   int bh, int sb, int qb, int lane) {
   constexpr int D = C::D;
-  constexpr int VPL = D / 32;
+  constexpr int VPL = D / 32;  // dimensions per lane
+  using V = VecOf<VPL>;
+  using VecT = typename V::T;
+  constexpr int G = 8;  // rows in flight per lane
   const int nKB = p.nKB;
   const float inv_sqrt_d = rsqrtf(static_cast<float>(D));
   const bool correct = (p.mode == 2);
   const int j0 = min((qb * C::BQ) / C::BK, nKB - 1);
-  const float *kb = p.kbar + static_cast<size_t>(bh) * nKB * D;
-  const float *vb = p.vbar + static_cast<size_t>(bh) * nKB * D;
+  const VecT *kb = reinterpret_cast<const VecT *>(p.kbar + static_cast<size_t>(bh) * nKB * D) + lane;
+  const VecT *vb = reinterpret_cast<const VecT *>(p.vbar + static_cast<size_t>(bh) * nKB * D) + lane;
   uint32_t *msk = sc.mask[sb];
-  const float4 *qv = reinterpret_cast<const float4 *>(sc.qrow);
 
+  float qv[VPL];
+  {
+    const float *qr = p.qbar + (static_cast<size_t>(bh) * p.nQB + qb) * D + lane * VPL;
+#pragma unroll
+    for (int e = 0; e < VPL; ++e) qv[e] = __ldg(qr + e);
+  }
   float M = -CUDART_INF_F;
   float cacc[VPL];
 #pragma unroll
@@ -164,25 +226,27 @@ __device__ __forceinline__ void route_query_block(SmemCtl<C> &sc, RouteSlot<C> &
   float lacc = 0.f;
 
   for (int t0 = 0; t0 < nKB; t0 += 32) {
+    float part[32];
+#pragma unroll
+    for (int g = 0; g < 32 / G; ++g) {
+      VecT kx[G];
+#pragma unroll
+      for (int e = 0; e < G; ++e) {
+        const int t = t0 + g * G + e;
+        int j = j0 + t;
+        if (j >= nKB) j -= nKB;
+        kx[e] = (t < nKB) ? __ldg(kb + static_cast<size_t>(j) * 32) : V::zero();
+      }
+#pragma unroll
+      for (int e = 0; e < G; ++e) part[g * G + e] = V::dot(qv, kx[e]);
+    }
     const int tt = t0 + lane;
     const bool valid = tt < nKB;
     int j = j0 + tt;
     if (j >= nKB) j -= nKB;
-    float s = -CUDART_INF_F;
-    if (valid) {
-      const float4 *kr = reinterpret_cast<const float4 *>(kb + static_cast<size_t>(j) * D);
-      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-#pragma unroll
-      for (int c = 0; c < D / 4; ++c) {
-        const float4 kx = __ldg(kr + c);
-        const float4 qx = qv[c];
-        a0 = fmaf(qx.x, kx.x, a0);
-        a1 = fmaf(qx.y, kx.y, a1);
-        a2 = fmaf(qx.z, kx.z, a2);
-        a3 = fmaf(qx.w, kx.w, a3);
-      }
-      s = ((a0 + a1) + (a2 + a3)) * inv_sqrt_d;
-    }
+    if (!valid) j = 0;
+    float s = warp_transpose_sum32(part, lane) * inv_sqrt_d;
+    if (!valid) s = -CUDART_INF_F;
     // Running maximum in visit order: inclusive prefix max over the lanes.
     float m = s;
 #pragma unroll
@@ -207,23 +271,24 @@ __device__ __forceinline__ void route_query_block(SmemCtl<C> &sc, RouteSlot<C> &
       const float w = drop ? nj * expf(s - M) : 0.f;
       lacc += w;
       uint32_t dm = __ballot_sync(0xffffffffu, drop);
-      while (dm) {
-        const int b = __ffs(dm) - 1;
-        dm &= dm - 1;
-        const float wb = __shfl_sync(0xffffffffu, w, b);
-        const int jb = __shfl_sync(0xffffffffu, j, b);
-        const float *vr = vb + static_cast<size_t>(jb) * D + lane * VPL;
-        if constexpr (VPL == 4) {
-          const float4 vv = __ldg(reinterpret_cast<const float4 *>(vr));
-          cacc[0] = fmaf(wb, vv.x, cacc[0]);
-          cacc[1] = fmaf(wb, vv.y, cacc[1]);
-          cacc[2] = fmaf(wb, vv.z, cacc[2]);
-          cacc[3] = fmaf(wb, vv.w, cacc[3]);
-        } else {
-          const float2 vv = __ldg(reinterpret_cast<const float2 *>(vr));
-          cacc[0] = fmaf(wb, vv.x, cacc[0]);
-          cacc[1] = fmaf(wb, vv.y, cacc[1]);
+      while (dm) {  // dm is warp-uniform
+        int src[G];
+#pragma unroll
+        for (int e = 0; e < G; ++e) {
+          src[e] = dm ? (__ffs(dm) - 1) : -1;
+          dm = dm ? (dm & (dm - 1)) : 0u;
         }
+        VecT vx[G];
+        float wb[G];
+#pragma unroll
+        for (int e = 0; e < G; ++e) {
+          const int b = src[e] < 0 ? 0 : src[e];
+          const int jb = __shfl_sync(0xffffffffu, j, b);
+          wb[e] = src[e] < 0 ? 0.f : __shfl_sync(0xffffffffu, w, b);
+          vx[e] = src[e] < 0 ? V::zero() : __ldg(vb + static_cast<size_t>(jb) * 32);
+        }
+#pragma unroll
+        for (int e = 0; e < G; ++e) V::axpy(cacc, wb[e], vx[e]);
       }
     } else {
       M = Mn;
@@ -280,9 +345,6 @@ __device__ void run_router(SmemCtl<C> &sc, const FwdParams &p, int lane) {
         }
         continue;
       }
-      const float *qr = p.qbar + (static_cast<size_t>(bh) * p.nQB + qb) * D;
-      for (int e = lane; e < D; e += 32) sc.qrow[e] = __ldg(qr + e);
-      __syncwarp();
       route_query_block<C>(sc, rs, p, bh, sb, qb, lane);
       __syncwarp();
     }
@@ -558,52 +620,56 @@ __device__ void run_softmax(SmemCtl<C> &sc, const FwdParams &p, uint32_t tmem, i
       const int j = rs.jlist[u];
       if (!wait(&sc.s_full[t], s_ph)) break;
       s_ph ^= 1;
-      uint32_t sr[BK / 32][32];
-#pragma unroll
-      for (int c = 0; c < BK / 32; ++c) tmem_ld32(s_addr + c * 32, sr[c]);
-      tmem_wait_ld();
-#pragma unroll
-      for (int c = 0; c < BK / 32; ++c) reg_fence32(sr[c]);
+      // S streams through registers 32 columns at a time; P is kept packed (fp16 pairs)
+      // until the whole row is done. The reference max only moves when a chunk exceeds
+      // it by more than the slack; then the P already packed is rescaled in registers.
       const bool rk = (mem & row_bit) != 0;
       const int ncol = (j == p.nKB - 1) ? (p.N - j * BK) : BK;
-      float mx = -CUDART_INF_F;
-      if (rk) {
+      float alpha = 1.f;  // total rescale of this row's O and l for this S tile
+      float lsum = 0.f;
+      uint32_t pk[BK / 2];
 #pragma unroll
-        for (int c = 0; c < BK / 32; ++c)
+      for (int c = 0; c < BK / 32; ++c) {
+        uint32_t sr[32];
+        tmem_ld32(s_addr + c * 32, sr);
+        tmem_wait_ld();
+        reg_fence32(sr);
+        float mx = -CUDART_INF_F;
+        if (rk) {
 #pragma unroll
           for (int e = 0; e < 32; ++e)
-            if (c * 32 + e < ncol) mx = fmaxf(mx, u2f(sr[c][e]));
-      }
-      const float mxs = mx * sc_log2;
-      float alpha = 1.f;
-      bool resc = false;
-      if (mxs > m_ref + kRescaleSlack) {
-        if (m_ref != -CUDART_INF_F) {
-          alpha = ex2_approx(m_ref - mxs);
-          resc = true;
+            if (c * 32 + e < ncol) mx = fmaxf(mx, u2f(sr[e]));
         }
-        m_ref = mxs;
-      }
-      l *= alpha;
-      const float neg_m = (m_ref == -CUDART_INF_F) ? 0.f : -m_ref;
-      float lsum = 0.f;
+        const float mxs = mx * sc_log2;
+        if (mxs > m_ref + kRescaleSlack) {
+          if (m_ref != -CUDART_INF_F) {
+            const float a = ex2_approx(m_ref - mxs);
+            alpha *= a;
+            lsum *= a;
+            const __half2 a2 = __float2half2_rn(a);
 #pragma unroll
-      for (int h = 0; h < BK / 64; ++h) {
-        uint32_t pk[32];
+            for (int e = 0; e < c * 16; ++e) {
+              __half2 h = *reinterpret_cast<__half2 *>(&pk[e]);
+              h = __hmul2(h, a2);
+              pk[e] = *reinterpret_cast<uint32_t *>(&h);
+            }
+          }
+          m_ref = mxs;
+        }
+        const float neg_m = (m_ref == -CUDART_INF_F) ? 0.f : -m_ref;
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int col = h * 64 + 2 * e;
-          const float x0 = u2f(sr[col >> 5][col & 31]);
-          const float x1 = u2f(sr[(col + 1) >> 5][(col + 1) & 31]);
-          const float p0 = (rk && col < ncol) ? ex2_approx(fmaf(x0, sc_log2, neg_m)) : 0.f;
-          const float p1 = (rk && col + 1 < ncol) ? ex2_approx(fmaf(x1, sc_log2, neg_m)) : 0.f;
+        for (int e = 0; e < 16; ++e) {
+          const int col = c * 32 + 2 * e;
+          const float p0 = (rk && col < ncol) ? ex2_approx(fmaf(u2f(sr[2 * e]), sc_log2, neg_m)) : 0.f;
+          const float p1 = (rk && col + 1 < ncol) ? ex2_approx(fmaf(u2f(sr[2 * e + 1]), sc_log2, neg_m)) : 0.f;
           lsum += p0 + p1;
-          pk[e] = pack_f16x2(p0, p1);
+          pk[c * 16 + e] = pack_f16x2(p0, p1);
         }
-        tmem_st32(s_addr + h * 32, pk);
       }
-      l += lsum;
-      if (__any_sync(0xffffffffu, resc)) {
+#pragma unroll
+      for (int h = 0; h < BK / 64; ++h) tmem_st32(s_addr + h * 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[h * 32]));
+      l = l * alpha + lsum;
+      if (__any_sync(0xffffffffu, alpha != 1.f)) {
         // The previous P V of this tile has completed (the commit that signalled this
         // S tile was issued after it), so O can be rescaled in place before the next one.
 #pragma unroll 1
