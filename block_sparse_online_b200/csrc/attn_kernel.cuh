@@ -49,6 +49,9 @@ constexpr float kLog2e = 1.4426950408889634f;
 // Lazy rescaling: a row's reference max moves only when the tile max exceeds it by
 // more than this many log2 units, so P stays <= 2^8 and O is rarely rescaled.
 constexpr float kRescaleSlack = 8.0f;
+// One pair of exponentials in this many is computed on the FMA pipe (polynomial)
+// instead of the MUFU unit, which the softmax otherwise saturates.
+constexpr int kPolyEvery = 4;
 
 struct FwdParams {
   int N;
@@ -620,54 +623,100 @@ __device__ void run_softmax(SmemCtl<C> &sc, const FwdParams &p, uint32_t tmem, i
       const int j = rs.jlist[u];
       if (!wait(&sc.s_full[t], s_ph)) break;
       s_ph ^= 1;
-      // S streams through registers 32 columns at a time; P is kept packed (fp16 pairs)
-      // until the whole row is done. The reference max only moves when a chunk exceeds
-      // it by more than the slack; then the P already packed is rescaled in registers.
+      // S streams through registers 64 columns (two 32-column loads, one wait) at a time
+      // and each 64-column half of P is stored to TMEM as soon as it is packed (fp16
+      // pairs). The reference max only moves when a half exceeds it by more than the
+      // slack; a half of P already stored is then rescaled in TMEM (rare).
       const bool rk = (mem & row_bit) != 0;
       const int ncol = (j == p.nKB - 1) ? (p.N - j * BK) : BK;
+      const bool full = rk && ncol == BK;  // warp-uniform: no column of this block masked
       float alpha = 1.f;  // total rescale of this row's O and l for this S tile
       float lsum = 0.f;
-      uint32_t pk[BK / 2];
 #pragma unroll
-      for (int c = 0; c < BK / 32; ++c) {
-        uint32_t sr[32];
-        tmem_ld32(s_addr + c * 32, sr);
+      for (int c2 = 0; c2 < BK / 64; ++c2) {
+        uint32_t sr[2][32];
+        tmem_ld32(s_addr + c2 * 64, sr[0]);
+        tmem_ld32(s_addr + c2 * 64 + 32, sr[1]);
         tmem_wait_ld();
-        reg_fence32(sr);
+        reg_fence32(sr[0]);
+        reg_fence32(sr[1]);
         float mx = -CUDART_INF_F;
-        if (rk) {
+        if (full) {
+          mx = fmax3(u2f(sr[0][0]), u2f(sr[0][1]), u2f(sr[0][2]));
 #pragma unroll
-          for (int e = 0; e < 32; ++e)
-            if (c * 32 + e < ncol) mx = fmaxf(mx, u2f(sr[e]));
+          for (int e = 3; e < 63; e += 2) mx = fmax3(mx, u2f(sr[e >> 5][e & 31]), u2f(sr[(e + 1) >> 5][(e + 1) & 31]));
+          mx = fmaxf(mx, u2f(sr[1][31]));
+        } else if (rk) {
+#pragma unroll
+          for (int e = 0; e < 64; ++e)
+            if (c2 * 64 + e < ncol) mx = fmaxf(mx, u2f(sr[e >> 5][e & 31]));
         }
         const float mxs = mx * sc_log2;
+        float a = 1.f;
         if (mxs > m_ref + kRescaleSlack) {
-          if (m_ref != -CUDART_INF_F) {
-            const float a = ex2_approx(m_ref - mxs);
-            alpha *= a;
-            lsum *= a;
-            const __half2 a2 = __float2half2_rn(a);
-#pragma unroll
-            for (int e = 0; e < c * 16; ++e) {
-              __half2 h = *reinterpret_cast<__half2 *>(&pk[e]);
-              h = __hmul2(h, a2);
-              pk[e] = *reinterpret_cast<uint32_t *>(&h);
-            }
-          }
+          if (m_ref != -CUDART_INF_F) a = ex2_approx(m_ref - mxs);
           m_ref = mxs;
         }
-        const float neg_m = (m_ref == -CUDART_INF_F) ? 0.f : -m_ref;
+        alpha *= a;
+        lsum *= a;
+        if (c2 > 0 && __any_sync(0xffffffffu, a != 1.f)) {
+          // Rescale the halves of P already in TMEM (their stores must land first).
+          tmem_wait_st();
+          const __half2 a2 = __float2half2_rn(a);
+#pragma unroll 1
+          for (int h = 0; h < c2; ++h) {
+            uint32_t pp[32];
+            tmem_ld32(s_addr + h * 32, pp);
+            tmem_wait_ld();
+            reg_fence32(pp);
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int col = c * 32 + 2 * e;
-          const float p0 = (rk && col < ncol) ? ex2_approx(fmaf(u2f(sr[2 * e]), sc_log2, neg_m)) : 0.f;
-          const float p1 = (rk && col + 1 < ncol) ? ex2_approx(fmaf(u2f(sr[2 * e + 1]), sc_log2, neg_m)) : 0.f;
-          lsum += p0 + p1;
-          pk[c * 16 + e] = pack_f16x2(p0, p1);
+            for (int e = 0; e < 32; ++e) {
+              __half2 v2 = *reinterpret_cast<__half2 *>(&pp[e]);
+              v2 = __hmul2(v2, a2);
+              pp[e] = *reinterpret_cast<uint32_t *>(&v2);
+            }
+            tmem_st32(s_addr + h * 32, pp);
+          }
         }
-      }
+        const float neg_m = (m_ref == -CUDART_INF_F) ? 0.f : -m_ref;
+        uint32_t pk[32];
+        if (full) {
+          // Packed fp32 pairs; one pair in kPolyEvery goes through the FMA-pipe exp2.
+          const uint64_t scp = f2(sc_log2, sc_log2);
+          const uint64_t nmp = f2(neg_m, neg_m);
+          uint64_t acc = f2(0.f, 0.f);
 #pragma unroll
-      for (int h = 0; h < BK / 64; ++h) tmem_st32(s_addr + h * 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[h * 32]));
+          for (int e = 0; e < 32; ++e) {
+            const uint64_t x = fma2(f2(u2f(sr[(2 * e) >> 5][(2 * e) & 31]), u2f(sr[(2 * e + 1) >> 5][(2 * e + 1) & 31])),
+                                    scp, nmp);
+            float x0, x1, p0, p1;
+            f2_split(x, x0, x1);
+            if ((e % kPolyEvery) == kPolyEvery - 1) {
+              exp2_poly_x2(x0, x1, p0, p1);
+            } else {
+              p0 = ex2_approx(x0);
+              p1 = ex2_approx(x1);
+            }
+            acc = add2(acc, f2(p0, p1));
+            pk[e] = pack_f16x2(p0, p1);
+          }
+          float s0, s1;
+          f2_split(acc, s0, s1);
+          lsum += s0 + s1;
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const int col = c2 * 64 + 2 * e;
+            const float x0 = u2f(sr[(2 * e) >> 5][(2 * e) & 31]);
+            const float x1 = u2f(sr[(2 * e + 1) >> 5][(2 * e + 1) & 31]);
+            const float p0 = (rk && col < ncol) ? ex2_approx(fmaf(x0, sc_log2, neg_m)) : 0.f;
+            const float p1 = (rk && col + 1 < ncol) ? ex2_approx(fmaf(x1, sc_log2, neg_m)) : 0.f;
+            lsum += p0 + p1;
+            pk[e] = pack_f16x2(p0, p1);
+          }
+        }
+        tmem_st32(s_addr + c2 * 32, pk);
+      }
       l = l * alpha + lsum;
       if (__any_sync(0xffffffffu, alpha != 1.f)) {
         // The previous P V of this tile has completed (the commit that signalled this
@@ -802,6 +851,17 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
     tc_fence_after_sync();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
+}
+
+// Evaluates the FMA-pipe exp2 used by the softmax on n inputs (self-test).
+__global__ void exp2_selftest_kernel(const float *x, float *y, int n) {
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i >= n) return;
+  const float x1 = (i + 1 < n) ? x[i + 1] : 0.f;
+  float y0, y1;
+  exp2_poly_x2(x[i], x1, y0, y1);
+  y[i] = y0;
+  if (i + 1 < n) y[i + 1] = y1;
 }
 
 // Device watchdog self-test: one thread waits on a barrier that nobody completes.

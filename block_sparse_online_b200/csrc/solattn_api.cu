@@ -341,6 +341,17 @@ int solattn_watchdog_selftest(void *workspace, size_t ws_bytes, uint64_t limit_n
   return cudaGetLastError() == cudaSuccess ? SOLATTN_OK : SOLATTN_ECUDA;
 }
 
+int solattn_selftest_exp2(const float *x, float *y, int n, void *stream) {
+  if (!x || !y || n < 0) return SOLATTN_EINVAL;
+  if (n == 0) return SOLATTN_OK;
+  DeviceInfo di;
+  if (device_info(&di) != SOLATTN_OK) return SOLATTN_ECUDA;
+  if (di.major != 10) return SOLATTN_EUNSUPPORTED;
+  const int pairs = (n + 1) / 2;
+  exp2_selftest_kernel<<<(pairs + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n);
+  return cudaGetLastError() == cudaSuccess ? SOLATTN_OK : SOLATTN_ECUDA;
+}
+
 const char *solattn_strerror(int status) {
   switch (status) {
     case SOLATTN_OK: return "ok";

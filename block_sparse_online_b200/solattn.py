@@ -29,7 +29,7 @@ MAX_KEY_BLOCKS = 1024
 EXPORTS = ("solattn_workspace_size", "solattn_pool", "solattn_forward", "solattn_forward_events",
            "solattn_get_status",
            "solattn_host_workspace_size", "solattn_forward_host", "solattn_watchdog_selftest",
-           "solattn_strerror")
+           "solattn_selftest_exp2", "solattn_strerror")
 
 
 class SolAttnError(RuntimeError):
@@ -64,6 +64,8 @@ def _load():
     lib.solattn_get_status.restype = i
     lib.solattn_watchdog_selftest.argtypes = [vp, sz, ctypes.c_uint64, vp]
     lib.solattn_watchdog_selftest.restype = i
+    lib.solattn_selftest_exp2.argtypes = [vp, vp, i, vp]
+    lib.solattn_selftest_exp2.restype = i
     lib.solattn_strerror.argtypes = [i]
     lib.solattn_strerror.restype = ctypes.c_char_p
     return lib
@@ -211,6 +213,16 @@ def solattn_watchdog_selftest(limit_ns: int = 2_000_000, stream=None) -> int:
     _check(_lib.solattn_watchdog_selftest(ws.data_ptr(), ws.numel(), int(limit_ns), _stream(stream)),
            "solattn_watchdog_selftest")
     return solattn_get_status(ws, stream)
+
+
+def solattn_selftest_exp2(x: torch.Tensor, stream=None) -> torch.Tensor:
+    """2^x by the software exp2 of the softmax, for a contiguous fp32 CUDA tensor."""
+    if x.dtype != torch.float32 or not x.is_cuda or not x.is_contiguous():
+        raise ValueError("x must be a contiguous fp32 CUDA tensor")
+    y = torch.empty_like(x)
+    _check(_lib.solattn_selftest_exp2(x.data_ptr(), y.data_ptr(), x.numel(), _stream(stream)),
+           "solattn_selftest_exp2")
+    return y
 
 
 __all__ = [n for n in globals() if n.startswith("solattn_")] + ["SolAttnError", "MODES"]

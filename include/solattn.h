@@ -167,6 +167,14 @@ int solattn_forward_host(const void *q, const void *k, const void *v, void *out,
 int solattn_watchdog_selftest(void *workspace, size_t ws_bytes, uint64_t limit_ns,
                               void *stream);
 
+/*
+ * Self-test of the software exp2 the softmax evaluates on the FMA pipe for part of
+ * its exponentials: y[i] = 2^x[i] for n device floats (x, y device pointers).
+ * Lets a test compare it with exp2 within its stated bound (relative error 7.5e-5
+ * for x >= -125; smaller inputs are clamped to -125).
+ */
+int solattn_selftest_exp2(const float *x, float *y, int n, void *stream);
+
 /* Static description of a status code. */
 const char *solattn_strerror(int status);
 

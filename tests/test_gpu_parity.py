@@ -157,3 +157,21 @@ def test_video720_config():
 @pytest.mark.slow
 def test_long_config():
     _full("long", (3.0, 4.0, 6.0, INF), MODES, per_head=2)
+
+
+def test_software_exp2_within_bound():
+    """The FMA-pipe exp2 of the softmax against fp64 2^x: relative error <= 7.5e-5 + fp32
+    rounding on the softmax's input range, and exact powers of two stay exact."""
+    from block_sparse_online_b200 import solattn
+    x = torch.cat([torch.linspace(-125.0, 8.0, 2_000_001), torch.arange(-125.0, 9.0),
+                   torch.rand(1_000_000) * 20 - 16]).contiguous()
+    y = solattn.solattn_selftest_exp2(x.cuda()).cpu().double().numpy()
+    want = np.exp2(x.double().numpy())
+    rel = np.abs(y - want) / want
+    assert rel.max() <= 7.6e-5, rel.max()
+    ints = torch.arange(-125.0, 9.0).double().numpy()
+    yi = solattn.solattn_selftest_exp2(torch.arange(-125.0, 9.0).cuda()).cpu().double().numpy()
+    np.testing.assert_allclose(yi, np.exp2(ints), rtol=7.6e-5)
+    # far below the clamp the result is a tiny positive number (zero once packed to fp16)
+    tiny = solattn.solattn_selftest_exp2(torch.tensor([-200.0, -1e30], device="cuda")).cpu()
+    assert (tiny >= 0).all() and (tiny < 1e-37).all()
