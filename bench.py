@@ -41,7 +41,7 @@ KERNEL_SOURCES = ["block_sparse_online_b200/csrc/attn_kernel.cuh", "block_sparse
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--config", default="video480")
@@ -118,20 +118,30 @@ class ClockSampler:
         self.lines = []
 
     def start(self):
+        """Start sampling every 50 ms and wait (up to 10 s) for the first sample, so the
+        samples taken afterwards cover the timed region."""
         try:
             self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
         except (OSError, ValueError):
             self.proc = None
+            return
+        t0 = time.time()
+        while not self.lines and time.time() - t0 < 10:
+            time.sleep(0.02)
+
+    def mark(self):
+        """Index of the next sample: samples from here on fall in the region being timed."""
+        return len(self.lines)
 
     def _read(self):
         for line in self.proc.stdout:
             self.lines.append(line.strip())
 
-    def stop(self):
+    def stop(self, first=0, last=None):
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         self.proc.terminate()
@@ -141,7 +151,7 @@ class ClockSampler:
             self.proc.kill()
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        for ln in self.lines[first:last]:
             f = [x.strip() for x in ln.split(",")]
             if len(f) < 9:
                 continue
@@ -198,6 +208,29 @@ def cores():
 
 
 # ------------------------------------------------------------------ main
+
+def rank_config(cfg, rank):
+    """Each rank of a multi-GPU run solves an independent problem of the same shape
+    (weak scaling): the same configuration with its own input seed."""
+    import dataclasses
+    return cfg if rank == 0 else dataclasses.replace(cfg, seed=cfg.seed + 7919 * rank)
+
+
+def max_over_ranks(x, world, device="cpu"):
+    """The largest value of x over the ranks (device times are reduced this way)."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(world, flops_per_rank, ms):
+    """Throughput of the whole job: the work all ranks did over the slowest rank's time."""
+    return world * flops_per_rank / (ms * 1e-3) / 1e12
+
 
 def dist_setup(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -257,12 +290,8 @@ def e2e_measure(args, cfg, q, k, v, dev, stream, world, barrier, dense_flops, el
                                      scratch=scratch)
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / e2e_steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    return {"value": round(world * dense_flops / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s (dense-equivalent)",
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world, dev)
+    return {"value": round(whole_job_rate(world, dense_flops, e2e_ms), 3), "unit": "TFLOP/s (dense-equivalent)",
             "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": 3 * elem * 2,
             "d2h_bytes_per_step": elem * 2 + B * H * 8, "steps": e2e_steps}
 
@@ -281,7 +310,7 @@ def main():
     dev = torch.device("cuda", local)
     if world > 1:
         dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
-    cfg = synth.CONFIGS[args.config]
+    cfg = rank_config(synth.CONFIGS[args.config], rank)
     if args.heads:
         import dataclasses
         cfg = dataclasses.replace(cfg, H=args.heads, note=cfg.note + f" [reduced to H={args.heads}]")
@@ -307,6 +336,7 @@ def main():
     dense_flops = cfg.dense_flops()
 
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    # (200 default steps of ~2 ms keep the timed region ~0.4 s: several 50 ms clock samples)
     ka = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     for _ in range(args.warmup):
         solattn.solattn_forward(qd, kd, vd, cfg.Bq, cfg.Bk, args.tau, args.mode, out=out, kept_per_head=kept,
@@ -314,9 +344,9 @@ def main():
     torch.cuda.synchronize()
     clocks = ClockSampler(local)
     clocks.start()
-    time.sleep(0.3)
     barrier()
     torch.cuda.synchronize()
+    first_sample = clocks.mark()
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     t_start.record(stream)
@@ -327,13 +357,10 @@ def main():
         ev[i][1].record(stream)
     t_end.record(stream)
     torch.cuda.synchronize()
+    last_sample = clocks.mark()
     barrier()
-    clk = clocks.stop()
-    total_ms = t_start.elapsed_time(t_end)
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    clk = clocks.stop(first_sample, max(last_sample, first_sample + 1))
+    total_ms = max_over_ranks(t_start.elapsed_time(t_end), world, dev)
     st = solattn.solattn_get_status(ws)
     if st != 0:
         raise RuntimeError(f"device status {st}")
@@ -341,7 +368,7 @@ def main():
     step_ms = [a.elapsed_time(b) for a, b in ev]
     attn_ms = [a.elapsed_time(b) for a, b in ka]
     attn_avg = sum(attn_ms) / len(attn_ms)
-    value = world * dense_flops / (ms_step * 1e-3) / 1e12
+    value = whole_job_rate(world, dense_flops, ms_step)
     peak_tf, peak_hbm, peak_kind = measured_peaks()
     achieved = exec_flops / (attn_avg * 1e-3) / 1e12
     trec = traffic_record()
