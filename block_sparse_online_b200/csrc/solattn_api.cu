@@ -159,6 +159,31 @@ int dispatch(int d, int Bq, int Bk, const CUtensorMap &mq, const CUtensorMap &mk
                    : dispatch_tiles<64, 64, 2>(mq, mk, mv, p, sms, st);
 }
 
+// ---- scratch for solattn_forward_noalloc
+//
+// A fixed device array, reserved when the library's module is loaded on a GPU and kept
+// until the process exits, so that callers who cannot allocate device memory still get
+// the operator's scratch (work counter, status word, pooled blocks, fp16 copy of V).
+// In host code `g_noalloc_scratch` is only a stand-in symbol: its device address is
+// looked up with cudaGetSymbolAddress, once per device, with that device current.
+constexpr size_t kNoAllocScratchBytes = SOLATTN_NOALLOC_SCRATCH_BYTES;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+void *g_noalloc_addr[64] = {};
+
+int noalloc_scratch(void **out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return SOLATTN_ECUDA;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_noalloc_addr[dev]) {
+    void *ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return SOLATTN_ECUDA;
+    g_noalloc_addr[dev] = ptr;
+  }
+  *out = g_noalloc_addr[dev];
+  return SOLATTN_OK;
+}
+
 int items_total(int B, int H, int N) {
   // Both tile shapes cover 2 x 128 query rows per work item.
   return B * H * ((N + 255) / 256);
@@ -278,6 +303,20 @@ int solattn_forward_events(const void *q, const void *k, const void *v, void *ou
                            size_t ws_bytes, void *stream, void *ev_attn_begin, void *ev_attn_end) {
   return forward_impl(q, k, v, out, B, H, N, d, Bq, Bk, tau, mode, stats, workspace, ws_bytes, stream,
                       ev_attn_begin, ev_attn_end);
+}
+
+int solattn_forward_noalloc(const void *q, const void *k, const void *v, void *out, int B, int H, int N, int d,
+                            int Bq, int Bk, float tau, int mode, const solattn_stats *stats, void *stream) {
+  const int rc = check_shape(B, H, N, d, Bq, Bk);
+  if (rc != SOLATTN_OK) return rc;
+  if (ws_layout(B, H, N, d, Bq, Bk).total > kNoAllocScratchBytes) return SOLATTN_EWORKSPACE;
+  void *scratch = nullptr;
+  const int rs = noalloc_scratch(&scratch);
+  if (rs != SOLATTN_OK) return rs;
+  // The forward path clears the scratch header (work counter, status word) on the
+  // stream before its kernels run, and overwrites every pooled block it reads.
+  return forward_impl(q, k, v, out, B, H, N, d, Bq, Bk, tau, mode, stats, scratch, kNoAllocScratchBytes, stream,
+                      nullptr, nullptr);
 }
 
 int solattn_get_status(const void *workspace, void *stream) {

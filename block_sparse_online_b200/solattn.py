@@ -29,7 +29,7 @@ MAX_KEY_BLOCKS = 1024
 EXPORTS = ("solattn_workspace_size", "solattn_pool", "solattn_forward", "solattn_forward_events",
            "solattn_get_status",
            "solattn_host_workspace_size", "solattn_forward_host", "solattn_watchdog_selftest",
-           "solattn_selftest_exp2", "solattn_strerror")
+           "solattn_selftest_exp2", "solattn_forward_noalloc", "solattn_strerror")
 
 
 class SolAttnError(RuntimeError):
@@ -64,6 +64,8 @@ def _load():
     lib.solattn_get_status.restype = i
     lib.solattn_watchdog_selftest.argtypes = [vp, sz, ctypes.c_uint64, vp]
     lib.solattn_watchdog_selftest.restype = i
+    lib.solattn_forward_noalloc.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, f, i, ctypes.POINTER(_Stats), vp]
+    lib.solattn_forward_noalloc.restype = i
     lib.solattn_selftest_exp2.argtypes = [vp, vp, i, vp]
     lib.solattn_selftest_exp2.restype = i
     lib.solattn_strerror.argtypes = [i]
@@ -213,6 +215,31 @@ def solattn_watchdog_selftest(limit_ns: int = 2_000_000, stream=None) -> int:
     _check(_lib.solattn_watchdog_selftest(ws.data_ptr(), ws.numel(), int(limit_ns), _stream(stream)),
            "solattn_watchdog_selftest")
     return solattn_get_status(ws, stream)
+
+
+NOALLOC_SCRATCH_BYTES = 64 << 20
+
+
+def solattn_forward_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, Bq: int, Bk: int, tau: float,
+                            mode="keep_correct", out: torch.Tensor | None = None,
+                            kept_per_head: torch.Tensor | None = None, stream=None):
+    """solattn_forward without a workspace: the library uses its static device scratch
+    (for callers that cannot allocate device memory). Output and count tensors are
+    allocated here only when not given; the library call itself allocates nothing.
+    Calls that overlap on the GPU race on the shared scratch."""
+    B, H, N, d = _bhnd(q)
+    for t in (q, k, v):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous() or tuple(t.shape) != (B, H, N, d):
+            raise ValueError("q, k, v must be contiguous bf16 CUDA tensors of one shape")
+    if out is None:
+        out = torch.empty_like(q)
+    if kept_per_head is None:
+        kept_per_head = torch.empty((B, H), dtype=torch.int64, device=q.device)
+    stats = _Stats(kept_per_head.data_ptr(), None)
+    rc = _lib.solattn_forward_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, H, N, d, Bq, Bk,
+                                      ctypes.c_float(float(tau)), _mode(mode), ctypes.byref(stats), _stream(stream))
+    _check(rc, "solattn_forward_noalloc")
+    return out, kept_per_head
 
 
 def solattn_selftest_exp2(x: torch.Tensor, stream=None) -> torch.Tensor:

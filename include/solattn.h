@@ -137,6 +137,42 @@ int solattn_forward_events(const void *q, const void *k, const void *v, void *ou
                            void *stream, void *ev_attn_begin, void *ev_attn_end);
 
 /*
+ * Size of the library's static device scratch used by solattn_forward_noalloc
+ * (64 MiB, held on every GPU that loads the library until the process exits).
+ */
+#define SOLATTN_NOALLOC_SCRATCH_BYTES (64u << 20)
+
+/*
+ * solattn_forward for callers that cannot allocate device memory. The paper has no
+ * counterpart to this entry point; it is an interface convenience of this library.
+ *
+ * Who needs it: code that receives only its input and output buffers and a stream
+ * (plugin interfaces of inference runtimes, callbacks that run while the host
+ * framework's allocator is locked, processes with a fixed device-memory budget where
+ * a late cudaMalloc fails or synchronises the whole device) cannot provide the
+ * workspace solattn_forward asks for. This entry point takes the same arguments minus
+ * the workspace and calls no allocating routine (no cudaMalloc, cudaFree or library
+ * allocator); its scratch is a static device array of SOLATTN_NOALLOC_SCRATCH_BYTES.
+ *
+ *   - The first call on a device looks up that array's device address
+ *     (cudaGetSymbolAddress) with the device current; make this first call before
+ *     any stream capture.
+ *   - Shapes whose solattn_workspace_size(...) exceeds SOLATTN_NOALLOC_SCRATCH_BYTES
+ *     are rejected with SOLATTN_EWORKSPACE before any device work.
+ *   - Every call on a device uses the same scratch, which keeps the previous call's
+ *     contents; the call clears what must start at zero (work counter, status word)
+ *     on its stream. Calls that overlap on the GPU (on different streams, or from
+ *     different threads) race on the scratch and give wrong results: serialise them.
+ *   - Device-side wait timeouts are recorded in the static scratch and are not
+ *     reported to the caller; use solattn_forward and solattn_get_status when that
+ *     status is needed.
+ * Arguments, results and the other errors are those of solattn_forward.
+ */
+int solattn_forward_noalloc(const void *q, const void *k, const void *v, void *out,
+                            int B, int H, int N, int d, int Bq, int Bk, float tau, int mode,
+                            const solattn_stats *stats, void *stream);
+
+/*
  * Synchronise `stream` and read the device status word of `workspace`
  * (SOLATTN_OK, or SOLATTN_ETIMEOUT if a bounded device-side wait gave up).
  */
