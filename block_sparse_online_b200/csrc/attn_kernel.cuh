@@ -1,19 +1,22 @@
 // attn_kernel.cuh -- the fused Sol-Attn forward kernel for sm_100a.
 //
-// One persistent CTA per SM processes work items. An item is NT = 2 adjacent
-// 128-row query tiles of one (batch, head) pair (each tile holds 128/Bq query
-// blocks). Roles, by warp:
-//   warp 0      TMA producer: Q tiles of the item, then K_j and V_j of every key
-//               block j in the item's kept list, into a ring of shared-memory slots.
-//   warp 1      MMA issuer (one thread): S_t = Q_t K_j^T into tensor memory (TMEM,
-//               bf16 -> fp32), O_t += P_t V_j with P_t read from TMEM (fp16 -> fp32).
+// One persistent CTA per SM processes work items. An item is one 128-row query tile
+// of one (batch, head) pair (the tile holds 128/Bq query blocks); its key stream is
+// the list of key blocks kept by any of the tile's query blocks. Roles, by warp:
+//   warp 0      TMA producer: the item's Q tile (double-buffered across items), then
+//               K_j and V_j of every kept block into a ring of shared-memory slots.
+//   warp 1      MMA issuer (one thread): S = Q K_j^T into tensor memory (TMEM,
+//               bf16 -> fp32), O += P V_j with P read from TMEM (fp16 -> fp32).
 //   warp 2      router: on-the-fly block thresholding and the correction sums for the
 //               NEXT item (double-buffered), from the fp32 pooled blocks in L2.
-//   warps 4..7  softmax warpgroup of tile 0, warps 8..11 of tile 1: online softmax
-//               with a lazily rescaled running max, P to TMEM, and the epilogue that
-//               merges the correction and writes bf16 rows.
-// The MMA warp interleaves the two tiles (ping-pong): while one warpgroup
-// exponentiates its S tile, the tensor core runs the other tile's P V and Q K^T.
+//   warps 4..7  softmax warpgroup A, warps 8..11 softmax warpgroup B. The tile's kept
+//               list is split between them (A takes entries 0, 2, 4, ..., B takes 1, 3,
+//               5, ...); each keeps its own S, O, running max and sum for all 128 rows.
+//               At the end of the item they exchange max and sum through shared memory
+//               and each writes half of the output columns of the merged result.
+// The MMA warp alternates A and B (ping-pong): while one warpgroup exponentiates its
+// S tile, the tensor core runs the other's P V and next Q K^T. Every K/V block is
+// loaded once.
 //
 // Method (paperlayer summary "Sol-Attn: Accelerating Video Generation Inference
 // via On-the-Fly Attention Sparsification", §3 Methodology):
@@ -72,33 +75,33 @@ struct FwdParams {
   unsigned long long timeout_ns;      // limit of every device-side wait
 };
 
-template <int D_, int BK_, int SUBQ_, int NT_>
+template <int D_, int BK_, int SUBQ_>
 struct Cfg {
   static constexpr int D = D_;
   static constexpr int BK = BK_;
   static constexpr int SUBQ = SUBQ_;  // query blocks per 128-row tile
-  static constexpr int NT = NT_;      // tiles per work item
   static constexpr int TILE_M = 128;
   static constexpr int BQ = TILE_M / SUBQ;
-  static constexpr int NSB = NT * SUBQ;  // query blocks per work item
+  static constexpr int NSB = SUBQ;       // query blocks per work item
   static constexpr int PANELS = D / 64;  // 128-byte swizzle panels per row
   static constexpr int Q_TILE_BYTES = TILE_M * D * 2;
+  static constexpr int NQBUF = 2;        // Q tiles in flight (current and next item)
   static constexpr int KV_BYTES = BK * D * 2;
   static constexpr int NSLOT = (131072 / KV_BYTES) < 8 ? (131072 / KV_BYTES) : 8;
-  static constexpr int TILE_COLS = BK + D;  // TMEM columns per tile: S (aliased by P) + O
-  static constexpr int TMEM_NEED = NT * TILE_COLS;
+  static constexpr int NWG = 2;              // softmax warpgroups sharing one tile
+  static constexpr int WG_COLS = BK + D;     // TMEM columns per warpgroup: S (aliased by P) + O
+  static constexpr int TMEM_NEED = NWG * WG_COLS;
   static constexpr int TMEM_COLS = TMEM_NEED <= 64 ? 64 : TMEM_NEED <= 128 ? 128 : TMEM_NEED <= 256 ? 256 : 512;
   // One control warpgroup (warp 0 producer, warp 1 MMA, warp 2 router, warp 3 spare)
-  // and one softmax warpgroup per tile. A warp may only touch TMEM lanes
-  // 32*(warp%4)..+31, so each softmax warpgroup covers the four lane quadrants once.
+  // and two softmax warpgroups. A warp may only touch TMEM lanes 32*(warp%4)..+31, so
+  // each softmax warpgroup covers the four lane quadrants once.
   static constexpr int CTRL_WARPS = 4;
-  static constexpr int NUM_THREADS = 32 * CTRL_WARPS + 128 * NT;
-  // Register split: the control warpgroup hands registers to the softmax warpgroups,
-  // which hold a whole S row. The sum stays within the registers the block is
-  // launched with (384 threads x 168).
+  static constexpr int NUM_THREADS = 32 * CTRL_WARPS + 128 * NWG;
+  // Register split: the control warpgroup hands registers to the softmax warpgroups.
+  // The sum stays within the registers the block is launched with (384 threads x 168).
   static constexpr int CTRL_REGS = 120;
   static constexpr int SOFTMAX_REGS = 192;
-  static_assert(NT != 2 || 128 * CTRL_REGS + 256 * SOFTMAX_REGS <= 384 * 168, "register split");
+  static_assert(128 * CTRL_REGS + 256 * SOFTMAX_REGS <= 384 * 168, "register split");
   // S = Q K^T in bf16; O += P V in fp16 (P in [0, 2^8] after the lazy rescale; V is the
   // fp16 copy written by the pooling pass).
   static constexpr uint32_t IDESC_QK = idesc_16bit_f32(128, BK, false, false);
@@ -123,10 +126,13 @@ template <class C>
 struct SmemCtl {
   RouteSlot<C> route[2];
   uint32_t mask[C::NSB][kMaskWords];  // router scratch: keep bits per query block
+  float xm[C::NWG][C::TILE_M];        // merge exchange: row max (log2 units) per warpgroup
+  float xl[C::NWG][C::TILE_M];        // merge exchange: row sum per warpgroup
   uint64_t full[C::NSLOT];
   uint64_t empty[C::NSLOT];
-  uint64_t q_full, q_empty;
-  uint64_t s_full[C::NT], p_full[C::NT], o_full[C::NT], o_empty[C::NT];
+  uint64_t q_full[C::NQBUF], q_empty[C::NQBUF];
+  uint64_t s_full[C::NWG], p_full[C::NWG], xchg[C::NWG];
+  uint64_t o_full, o_empty;
   uint64_t route_full[2], route_empty[2];
   uint64_t mma_done;
   uint32_t tmem_base;
@@ -135,7 +141,7 @@ struct SmemCtl {
 
 template <class C>
 constexpr size_t fwd_smem_bytes() {
-  return 1024 + static_cast<size_t>(C::NT) * C::Q_TILE_BYTES +
+  return 1024 + static_cast<size_t>(C::NQBUF) * C::Q_TILE_BYTES +
          static_cast<size_t>(C::NSLOT) * C::KV_BYTES + sizeof(SmemCtl<C>);
 }
 
@@ -415,6 +421,22 @@ __device__ void run_producer(SmemCtl<C> &sc, const FwdParams &p, uint8_t *q_smem
   const volatile int *ab = &sc.abort_flag;
   uint32_t kv_it = 0, q_it = 0;
   bool ok = true;
+  // Loads one K or V tile of key block j into the next ring slot.
+  auto load = [&](int j, bool is_v, int bh) {
+    const int slot = kv_it % C::NSLOT;
+    const uint32_t ph = (kv_it / C::NSLOT) & 1;
+    if (!mbar_wait(&sc.empty[slot], ph ^ 1, p.timeout_ns, ab)) {
+      ok = false;
+      return;
+    }
+    mbar_arrive_expect_tx(&sc.full[slot], C::KV_BYTES);
+    uint8_t *dst = ring + slot * C::KV_BYTES;
+#pragma unroll
+    for (int pn = 0; pn < C::PANELS; ++pn)
+      tma_load_3d(smem_u32(dst + pn * (C::BK * 128)), is_v ? tm_v : tm_k, smem_u32(&sc.full[slot]), pn * 64,
+                  j * C::BK, bh);
+    ++kv_it;
+  };
   for (uint32_t r_it = 0;; ++r_it) {
     const int s = r_it & 1;
     if (!mbar_wait(&sc.route_full[s], (r_it >> 1) & 1, p.timeout_ns, ab)) { ok = false; break; }
@@ -422,50 +444,41 @@ __device__ void run_producer(SmemCtl<C> &sc, const FwdParams &p, uint8_t *q_smem
     const int item = rs.item;
     if (item < 0) break;
     const int bh = item / p.items_per_head;
-    const int row0 = (item - bh * p.items_per_head) * (C::NT * C::TILE_M);
-    if (!mbar_wait(&sc.q_empty, (q_it & 1) ^ 1, p.timeout_ns, ab)) { ok = false; break; }
-    mbar_arrive_expect_tx(&sc.q_full, C::NT * C::Q_TILE_BYTES);
+    const int row0 = (item - bh * p.items_per_head) * C::TILE_M;
+    const int qb = q_it & 1;
+    if (!mbar_wait(&sc.q_empty[qb], ((q_it >> 1) & 1) ^ 1, p.timeout_ns, ab)) { ok = false; break; }
+    mbar_arrive_expect_tx(&sc.q_full[qb], C::Q_TILE_BYTES);
 #pragma unroll
-    for (int t = 0; t < C::NT; ++t)
-#pragma unroll
-      for (int pn = 0; pn < C::PANELS; ++pn)
-        tma_load_3d(smem_u32(q_smem + t * C::Q_TILE_BYTES + pn * (C::TILE_M * 128)), tm_q,
-                    smem_u32(&sc.q_full), pn * 64, row0 + t * C::TILE_M, bh);
+    for (int pn = 0; pn < C::PANELS; ++pn)
+      tma_load_3d(smem_u32(q_smem + qb * C::Q_TILE_BYTES + pn * (C::TILE_M * 128)), tm_q, smem_u32(&sc.q_full[qb]),
+                  pn * 64, row0, bh);
     ++q_it;
+    // Ring order = consumption order of the MMA warp: K_0, K_1, then V_u, K_{u+2}.
     const int n = rs.n_union;
+    load(rs.jlist[0], false, bh);
+    if (ok && n > 1) load(rs.jlist[1], false, bh);
     for (int u = 0; u < n && ok; ++u) {
-      const int j = rs.jlist[u];
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        const int slot = kv_it % C::NSLOT;
-        const uint32_t ph = (kv_it / C::NSLOT) & 1;
-        if (!mbar_wait(&sc.empty[slot], ph ^ 1, p.timeout_ns, ab)) { ok = false; break; }
-        mbar_arrive_expect_tx(&sc.full[slot], C::KV_BYTES);
-        uint8_t *dst = ring + slot * C::KV_BYTES;
-#pragma unroll
-        for (int pn = 0; pn < C::PANELS; ++pn)
-          tma_load_3d(smem_u32(dst + pn * (C::BK * 128)), half ? tm_v : tm_k, smem_u32(&sc.full[slot]),
-                      pn * 64, j * C::BK, bh);
-        ++kv_it;
-      }
+      load(rs.jlist[u], true, bh);
+      if (ok && u + 2 < n) load(rs.jlist[u + 2], false, bh);
     }
     if (!ok) break;
     mbar_arrive(&sc.route_empty[s]);
   }
   if (!ok) raise_abort(&sc.abort_flag, p.status);
   // No copy may outlive the block: wait (bounded, ignoring the abort flag) for the
-  // last fill of every slot and of the Q tiles to land.
+  // last fill of every slot and of the Q buffers to land.
   const int zero = 0;
   for (uint32_t f = (kv_it > C::NSLOT ? kv_it - C::NSLOT : 0); f < kv_it; ++f)
     mbar_wait(&sc.full[f % C::NSLOT], (f / C::NSLOT) & 1, p.timeout_ns, &zero);
-  if (q_it > 0) mbar_wait(&sc.q_full, (q_it - 1) & 1, p.timeout_ns, &zero);
+  for (uint32_t f = (q_it > C::NQBUF ? q_it - C::NQBUF : 0); f < q_it; ++f)
+    mbar_wait(&sc.q_full[f & 1], (f >> 1) & 1, p.timeout_ns, &zero);
 }
 
 // ------------------------------------------------------------------ MMA issuer
 
 template <class C>
-__device__ __forceinline__ void issue_qk(uint32_t tmem, int t, uint32_t q_base, uint32_t k_base) {
-  const uint32_t d_tmem = tmem + t * C::TILE_COLS;
+__device__ __forceinline__ void issue_qk(uint32_t tmem, int w, uint32_t q_base, uint32_t k_base) {
+  const uint32_t d_tmem = tmem + w * C::WG_COLS;
 #pragma unroll
   for (int kk = 0; kk < C::D / 16; ++kk) {
     const uint32_t off_q = (kk >> 2) * (C::TILE_M * 128) + (kk & 3) * 32;
@@ -476,9 +489,9 @@ __device__ __forceinline__ void issue_qk(uint32_t tmem, int t, uint32_t q_base, 
 }
 
 template <class C>
-__device__ __forceinline__ void issue_pv(uint32_t tmem, int t, uint32_t v_base, bool accumulate) {
-  const uint32_t d_tmem = tmem + t * C::TILE_COLS + C::BK;
-  const uint32_t p_tmem = tmem + t * C::TILE_COLS;
+__device__ __forceinline__ void issue_pv(uint32_t tmem, int w, uint32_t v_base, bool accumulate) {
+  const uint32_t d_tmem = tmem + w * C::WG_COLS + C::BK;
+  const uint32_t p_tmem = tmem + w * C::WG_COLS;
 #pragma unroll
   for (int kk = 0; kk < C::BK / 16; ++kk) {
     mma_bf16_ts(d_tmem, p_tmem + kk * 8, smem_desc_sw128(v_base + kk * (16 * 128), C::BK * 128, 1024),
@@ -491,17 +504,21 @@ __device__ void run_mma(SmemCtl<C> &sc, const FwdParams &p, uint32_t tmem, uint8
   const volatile int *ab = &sc.abort_flag;
   const uint32_t q_base = smem_u32(q_smem);
   const uint32_t ring_base = smem_u32(ring);
-  constexpr uint32_t TILE_BITS = (1u << C::SUBQ) - 1u;
   uint32_t kv_it = 0, q_it = 0, o_it = 0;
-  uint32_t p_ph[C::NT];
-#pragma unroll
-  for (int t = 0; t < C::NT; ++t) p_ph[t] = 0;
+  uint32_t p_ph[C::NWG] = {0, 0};
   bool ok = true;
   auto wait = [&](uint64_t *bar, uint32_t par) {
     if (!ok) return false;
     if (!mbar_wait(bar, par, p.timeout_ns, ab)) ok = false;
     else tc_fence_after_sync();
     return ok;
+  };
+  // Next ring slot, once its copy has landed (-1 on timeout).
+  auto next_slot = [&]() {
+    const int slot = kv_it % C::NSLOT;
+    if (!wait(&sc.full[slot], (kv_it / C::NSLOT) & 1)) return -1;
+    ++kv_it;
+    return slot;
   };
   for (uint32_t r_it = 0; ok; ++r_it) {
     const int s = r_it & 1;
@@ -510,65 +527,41 @@ __device__ void run_mma(SmemCtl<C> &sc, const FwdParams &p, uint32_t tmem, uint8
     const int item = rs.item;
     if (item < 0) break;
     const int n = rs.n_union;
-    if (!wait(&sc.q_full, q_it & 1)) break;
+    const int qb = q_it & 1;
+    if (!wait(&sc.q_full[qb], (q_it >> 1) & 1)) break;
     ++q_it;
-    // prologue: S for the first kept key block
-    int kslot = kv_it % C::NSLOT;
-    if (!wait(&sc.full[kslot], (kv_it / C::NSLOT) & 1)) break;
-    ++kv_it;
-    uint32_t mem = rs.member[0];
-#pragma unroll
-    for (int t = 0; t < C::NT; ++t)
-      if ((mem >> (t * C::SUBQ)) & TILE_BITS) {
-        issue_qk<C>(tmem, t, q_base + t * C::Q_TILE_BYTES, ring_base + kslot * C::KV_BYTES);
-        tc_commit(&sc.s_full[t]);
-      }
-    tc_commit(&sc.empty[kslot]);
-    if (n == 1) tc_commit(&sc.q_empty);
-    bool first[C::NT];
-#pragma unroll
-    for (int t = 0; t < C::NT; ++t) first[t] = true;
+    const uint32_t q_addr = q_base + qb * C::Q_TILE_BYTES;
+    // Prologue: S for the first kept block of each warpgroup.
+    for (int u0 = 0; u0 < n && u0 < 2; ++u0) {
+      const int ks = next_slot();
+      if (ks < 0) break;
+      issue_qk<C>(tmem, u0, q_addr, ring_base + ks * C::KV_BYTES);
+      tc_commit(&sc.s_full[u0]);
+      tc_commit(&sc.empty[ks]);
+    }
+    if (!ok) break;
+    if (n <= 2) tc_commit(&sc.q_empty[qb]);
     for (int u = 0; u < n && ok; ++u) {
-      const int vslot = kv_it % C::NSLOT;
-      if (!wait(&sc.full[vslot], (kv_it / C::NSLOT) & 1)) break;
-      ++kv_it;
-      const bool has_next = (u + 1) < n;
-      uint32_t memn = 0;
-      if (has_next) {
-        kslot = kv_it % C::NSLOT;
-        if (!wait(&sc.full[kslot], (kv_it / C::NSLOT) & 1)) break;
-        ++kv_it;
-        memn = rs.member[u + 1];
+      const int w = u & 1;
+      const int vs = next_slot();
+      if (vs < 0) break;
+      if (!wait(&sc.p_full[w], p_ph[w])) break;
+      p_ph[w] ^= 1;
+      // The first P V of the item overwrites O: the previous item's epilogue must be done.
+      if (u == 0 && !wait(&sc.o_empty, (o_it & 1) ^ 1)) break;
+      issue_pv<C>(tmem, w, ring_base + vs * C::KV_BYTES, u >= 2);
+      tc_commit(&sc.empty[vs]);
+      if (u + 2 < n) {
+        const int ks = next_slot();
+        if (ks < 0) break;
+        issue_qk<C>(tmem, w, q_addr, ring_base + ks * C::KV_BYTES);
+        tc_commit(&sc.s_full[w]);
+        tc_commit(&sc.empty[ks]);
+        if (u + 2 == n - 1) tc_commit(&sc.q_empty[qb]);
       }
-#pragma unroll
-      for (int t = 0; t < C::NT; ++t) {
-        if ((mem >> (t * C::SUBQ)) & TILE_BITS) {
-          if (!wait(&sc.p_full[t], p_ph[t])) break;
-          p_ph[t] ^= 1;
-          if (first[t] && !wait(&sc.o_empty[t], (o_it & 1) ^ 1)) break;
-          issue_pv<C>(tmem, t, ring_base + vslot * C::KV_BYTES, !first[t]);
-          first[t] = false;
-        }
-        if ((memn >> (t * C::SUBQ)) & TILE_BITS) {
-          issue_qk<C>(tmem, t, q_base + t * C::Q_TILE_BYTES, ring_base + kslot * C::KV_BYTES);
-          tc_commit(&sc.s_full[t]);
-        }
-      }
-      if (!ok) break;
-      tc_commit(&sc.empty[vslot]);
-      if (has_next) {
-        tc_commit(&sc.empty[kslot]);
-        if (u + 2 == n) tc_commit(&sc.q_empty);
-      }
-      mem = memn;
     }
     if (!ok) break;
-#pragma unroll
-    for (int t = 0; t < C::NT; ++t) {
-      if (first[t] && !wait(&sc.o_empty[t], (o_it & 1) ^ 1)) break;
-      tc_commit(&sc.o_full[t]);
-    }
-    if (!ok) break;
+    tc_commit(&sc.o_full);
     ++o_it;
     mbar_arrive(&sc.route_empty[s]);
   }
@@ -582,27 +575,26 @@ __device__ void run_mma(SmemCtl<C> &sc, const FwdParams &p, uint32_t tmem, uint8
 // ------------------------------------------------------------------ softmax / epilogue
 
 template <class C>
-__device__ void run_softmax(SmemCtl<C> &sc, const FwdParams &p, uint32_t tmem, int t, int warp, int lane) {
+__device__ void run_softmax(SmemCtl<C> &sc, const FwdParams &p, uint32_t tmem, int w, int warp, int lane) {
   constexpr int BK = C::BK;
   constexpr int D = C::D;
-  constexpr uint32_t TILE_BITS = ((1u << C::SUBQ) - 1u);
   const volatile int *ab = &sc.abort_flag;
   const int wq = warp & 3;  // TMEM lane quadrant this warp may access
   const int row = wq * 32 + lane;
-  const uint32_t s_addr = tmem + (static_cast<uint32_t>(wq * 32) << 16) + t * C::TILE_COLS;
+  const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+  const uint32_t s_addr = lane_base + w * C::WG_COLS;
   const uint32_t o_addr = s_addr + BK;
   const float sc_log2 = kLog2e * rsqrtf(static_cast<float>(D));
-  const int sb = t * C::SUBQ + (C::SUBQ == 2 ? (row >> 6) : 0);
+  const int sb = (C::SUBQ == 2 ? (row >> 6) : 0);
   const uint32_t row_bit = 1u << sb;
-  const uint32_t tile_bits = TILE_BITS << (t * C::SUBQ);
   uint32_t s_ph = 0;
   bool ok = true;
   auto wait = [&](uint64_t *bar, uint32_t par) {
-    bool w = mbar_wait(bar, par, p.timeout_ns, ab);
-    w = __all_sync(0xffffffffu, w);
-    if (!w) ok = false;
+    bool wt = mbar_wait(bar, par, p.timeout_ns, ab);
+    wt = __all_sync(0xffffffffu, wt);
+    if (!wt) ok = false;
     else tc_fence_after_sync();
-    return w;
+    return wt;
   };
   for (uint32_t r_it = 0; ok; ++r_it) {
     const int s = r_it & 1;
@@ -611,17 +603,15 @@ __device__ void run_softmax(SmemCtl<C> &sc, const FwdParams &p, uint32_t tmem, i
     const int item = rs.item;
     if (item < 0) break;
     const int bh = item / p.items_per_head;
-    const int pidx = item - bh * p.items_per_head;
-    const int grow = pidx * (C::NT * C::TILE_M) + t * C::TILE_M + row;
+    const int tile = item - bh * p.items_per_head;
+    const int grow = tile * C::TILE_M + row;
     const int n = rs.n_union;
     float m_ref = -CUDART_INF_F;  // reference max of this row, log2 units
     float l = 0.f;
-    bool any = false;
-    for (int u = 0; u < n; ++u) {
+    for (int u = w; u < n; u += 2) {
       const uint32_t mem = rs.member[u];
-      if (!(mem & tile_bits)) continue;
       const int j = rs.jlist[u];
-      if (!wait(&sc.s_full[t], s_ph)) break;
+      if (!wait(&sc.s_full[w], s_ph)) break;
       s_ph ^= 1;
       // S streams through registers 64 columns (two 32-column loads, one wait) at a time
       // and each 64-column half of P is stored to TMEM as soon as it is packed (fp16
@@ -719,7 +709,7 @@ __device__ void run_softmax(SmemCtl<C> &sc, const FwdParams &p, uint32_t tmem, i
       }
       l = l * alpha + lsum;
       if (__any_sync(0xffffffffu, alpha != 1.f)) {
-        // The previous P V of this tile has completed (the commit that signalled this
+        // The previous P V of this warpgroup has completed (the commit that signalled this
         // S tile was issued after it), so O can be rescaled in place before the next one.
 #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
@@ -734,48 +724,62 @@ __device__ void run_softmax(SmemCtl<C> &sc, const FwdParams &p, uint32_t tmem, i
       }
       tmem_wait_st();
       tc_fence_before_sync();
-      mbar_arrive(&sc.p_full[t]);
-      any = true;
+      mbar_arrive(&sc.p_full[w]);
     }
     if (!ok) break;
-    // Epilogue: O / l merged with the correction of this row's query block.
-    if (!wait(&sc.o_full[t], r_it & 1)) break;
-    if (any) {
-      const int qb = pidx * C::NSB + sb;
-      const bool valid = (grow < p.N) && (qb < p.nQB);
-      float a = 1.f, b = 0.f;
-      const float Lc = rs.L[sb];
-      if (Lc > 0.f) {
-        const float M2 = rs.M[sb] * kLog2e;
-        const float Ms = fmaxf(m_ref, M2);
-        a = ex2_approx(m_ref - Ms);
-        b = ex2_approx(M2 - Ms);
-      }
-      const float inv = 1.f / (a * l + b * Lc);
-      const float *cv = rs.Cv[sb];
-      uint4 *dst = reinterpret_cast<uint4 *>(p.out + (static_cast<size_t>(bh) * p.N + grow) * D);
+    // Epilogue: wait for the last P V of both warpgroups, exchange the row max and sum,
+    // and write this warpgroup's half of the output columns of the merged rows.
+    if (!wait(&sc.o_full, r_it & 1)) break;
+    sc.xm[w][row] = m_ref;
+    sc.xl[w][row] = l;
+    mbar_arrive(&sc.xchg[w]);
+    if (!wait(&sc.xchg[w ^ 1], r_it & 1)) break;
+    const float mA = sc.xm[0][row], lA = sc.xl[0][row];
+    const float mB = sc.xm[1][row], lB = sc.xl[1][row];
+    const bool hasB = n >= 2;  // warpgroup B ran at least one P V (A always does)
+    const int qb = tile * C::NSB + sb;
+    const bool valid = (grow < p.N) && (qb < p.nQB);
+    const float Lc = rs.L[sb];
+    const float M2 = rs.M[sb] * kLog2e;
+    float Ms = -CUDART_INF_F;
+    if (lA > 0.f) Ms = mA;
+    if (hasB && lB > 0.f) Ms = fmaxf(Ms, mB);
+    if (Lc > 0.f) Ms = fmaxf(Ms, M2);
+    const float aA = (lA > 0.f) ? ex2_approx(mA - Ms) : 0.f;
+    const float aB = (hasB && lB > 0.f) ? ex2_approx(mB - Ms) : 0.f;
+    const float b = (Lc > 0.f) ? ex2_approx(M2 - Ms) : 0.f;
+    const float inv = 1.f / (aA * lA + aB * lB + b * Lc);
+    const float *cv = rs.Cv[sb];
+    const uint32_t oA = lane_base + C::BK;
+    const uint32_t oB = lane_base + C::WG_COLS + C::BK;
+    uint4 *dst = reinterpret_cast<uint4 *>(p.out + (static_cast<size_t>(bh) * p.N + grow) * D);
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t o[32];
-        tmem_ld32(o_addr + c * 32, o);
-        tmem_wait_ld();
-        reg_fence32(o);
-        if (valid) {
-          uint32_t pk[16];
+    for (int c = 0; c < D / 32; ++c) {
+      const int col0 = w * (D / 2) + c * 16;
+      uint32_t xa[16], xb[16];
+      tmem_ld16(oA + col0, xa);
+      if (hasB) tmem_ld16(oB + col0, xb);
+      tmem_wait_ld();
+      reg_fence16(xa);
+      reg_fence16(xb);
+      if (valid) {
+        uint32_t pk[8];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const float y0 = fmaf(a, u2f(o[2 * e]), b * cv[c * 32 + 2 * e]) * inv;
-            const float y1 = fmaf(a, u2f(o[2 * e + 1]), b * cv[c * 32 + 2 * e + 1]) * inv;
-            pk[e] = pack_bf16x2(y0, y1);
+        for (int e = 0; e < 8; ++e) {
+          float y0 = fmaf(aA, u2f(xa[2 * e]), b * cv[col0 + 2 * e]);
+          float y1 = fmaf(aA, u2f(xa[2 * e + 1]), b * cv[col0 + 2 * e + 1]);
+          if (hasB) {
+            y0 = fmaf(aB, u2f(xb[2 * e]), y0);
+            y1 = fmaf(aB, u2f(xb[2 * e + 1]), y1);
           }
-#pragma unroll
-          for (int v = 0; v < 4; ++v)
-            dst[c * 4 + v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+          pk[e] = pack_bf16x2(y0 * inv, y1 * inv);
         }
+        dst[(col0 >> 3)] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        dst[(col0 >> 3) + 1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
       }
     }
     tc_fence_before_sync();
-    mbar_arrive(&sc.o_empty[t]);
+    mbar_arrive(&sc.o_empty);
     mbar_arrive(&sc.route_empty[s]);
   }
   if (!ok && lane == 0) raise_abort(&sc.abort_flag, p.status);
@@ -790,7 +794,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *q_smem = base;
-  uint8_t *ring = base + C::NT * C::Q_TILE_BYTES;
+  uint8_t *ring = base + C::NQBUF * C::Q_TILE_BYTES;
   SmemCtl<C> &sc = *reinterpret_cast<SmemCtl<C> *>(ring + C::NSLOT * C::KV_BYTES);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -800,17 +804,20 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
       mbar_init(&sc.full[i], 1);
       mbar_init(&sc.empty[i], 1);
     }
-    mbar_init(&sc.q_full, 1);
-    mbar_init(&sc.q_empty, 1);
-    for (int t = 0; t < C::NT; ++t) {
-      mbar_init(&sc.s_full[t], 1);
-      mbar_init(&sc.p_full[t], 128);
-      mbar_init(&sc.o_full[t], 1);
-      mbar_init(&sc.o_empty[t], 128);
+    for (int i = 0; i < C::NQBUF; ++i) {
+      mbar_init(&sc.q_full[i], 1);
+      mbar_init(&sc.q_empty[i], 1);
     }
+    for (int w = 0; w < C::NWG; ++w) {
+      mbar_init(&sc.s_full[w], 1);
+      mbar_init(&sc.p_full[w], 128);
+      mbar_init(&sc.xchg[w], 128);
+    }
+    mbar_init(&sc.o_full, 1);
+    mbar_init(&sc.o_empty, 128 * C::NWG);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&sc.route_full[s], 1);
-      mbar_init(&sc.route_empty[s], 2 + 128 * C::NT);
+      mbar_init(&sc.route_empty[s], 2 + 128 * C::NWG);
     }
     mbar_init(&sc.mma_done, 1);
     sc.abort_flag = 0;

@@ -139,8 +139,8 @@ int launch_fwd(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &
 template <int D, int BK, int SUBQ>
 int dispatch_tiles(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv, FwdParams p, int sms,
                    cudaStream_t st) {
-  using C = Cfg<D, BK, SUBQ, 2>;
-  p.items_per_head = (p.N + C::NT * C::TILE_M - 1) / (C::NT * C::TILE_M);
+  using C = Cfg<D, BK, SUBQ>;
+  p.items_per_head = (p.N + C::TILE_M - 1) / C::TILE_M;
   return launch_fwd<C>(mq, mk, mv, p, sms, st);
 }
 
@@ -185,8 +185,8 @@ int noalloc_scratch(void **out) {
 }
 
 int items_total(int B, int H, int N) {
-  // Both tile shapes cover 2 x 128 query rows per work item.
-  return B * H * ((N + 255) / 256);
+  // One work item per 128-row query tile.
+  return B * H * ((N + 127) / 128);
 }
 
 int forward_impl(const void *q, const void *k, const void *v, void *out, int B, int H, int N, int d, int Bq, int Bk,
