@@ -71,6 +71,7 @@ struct FwdParams {
   unsigned long long *kept_per_head;  // [BH]
   uint32_t *keep_mask;                // [BH][nQB][ceil(nKB/32)] or null
   unsigned int *counter;              // work-item counter, zero at launch
+  const int *order;                   // fetch order of the work items, or null (item order)
   int *status;                        // device status word
   unsigned long long timeout_ns;      // limit of every device-side wait
 };
@@ -202,25 +203,25 @@ struct VecOf<2> {
 };
 
 // Route one query block: visit its key blocks in order, keep those whose proxy clears
-// the running maximum minus tau, and (keep_correct) fold every dropped block into the
-// correction sums. Lane-per-dimension layout: each pooled row is one coalesced
-// 128/256-byte load across the warp, loads are issued 8 rows at a time, and the 32
-// per-block dot products of a chunk are finished with one transpose-sum.
-template <class C>
-__device__ __forceinline__ void route_query_block(SmemCtl<C> &sc, RouteSlot<C> &rs, const FwdParams &p,
-                                                  int bh, int sb, int qb, int lane) {
-  constexpr int D = C::D;
+// the running maximum minus tau, and (if `correct`) fold every dropped block into the
+// correction sums (cacc, lacc relative to the running max M). Keep bits are OR-ed into
+// `msk` (shared memory, zeroed by the caller). Lane-per-dimension layout: each pooled
+// row is one coalesced 128/256-byte load across the warp, loads are issued 8 rows at a
+// time, and the 32 per-block dot products of a chunk are finished with one
+// transpose-sum. The attention kernel's router and the planning kernel both route
+// through this function, so they take identical decisions.
+template <int D, int BQ, int BK>
+__device__ __forceinline__ void route_scan(const FwdParams &p, int bh, int qb, int lane, bool correct, uint32_t *msk,
+                                           float (&cacc)[D / 32], float &lacc, float &M) {
   constexpr int VPL = D / 32;  // dimensions per lane
   using V = VecOf<VPL>;
   using VecT = typename V::T;
   constexpr int G = 8;  // rows in flight per lane
   const int nKB = p.nKB;
   const float inv_sqrt_d = rsqrtf(static_cast<float>(D));
-  const bool correct = (p.mode == 2);
-  const int j0 = min((qb * C::BQ) / C::BK, nKB - 1);
+  const int j0 = min((qb * BQ) / BK, nKB - 1);
   const VecT *kb = reinterpret_cast<const VecT *>(p.kbar + static_cast<size_t>(bh) * nKB * D) + lane;
   const VecT *vb = reinterpret_cast<const VecT *>(p.vbar + static_cast<size_t>(bh) * nKB * D) + lane;
-  uint32_t *msk = sc.mask[sb];
 
   float qv[VPL];
   {
@@ -228,11 +229,10 @@ __device__ __forceinline__ void route_query_block(SmemCtl<C> &sc, RouteSlot<C> &
 #pragma unroll
     for (int e = 0; e < VPL; ++e) qv[e] = __ldg(qr + e);
   }
-  float M = -CUDART_INF_F;
-  float cacc[VPL];
+  M = -CUDART_INF_F;
 #pragma unroll
   for (int e = 0; e < VPL; ++e) cacc[e] = 0.f;
-  float lacc = 0.f;
+  lacc = 0.f;
 
   for (int t0 = 0; t0 < nKB; t0 += 32) {
     float part[32];
@@ -276,7 +276,7 @@ __device__ __forceinline__ void route_query_block(SmemCtl<C> &sc, RouteSlot<C> &
         M = Mn;
       }
       const bool drop = valid && !keep;
-      const float nj = (j == nKB - 1) ? static_cast<float>(p.N - j * C::BK) : static_cast<float>(C::BK);
+      const float nj = (j == nKB - 1) ? static_cast<float>(p.N - j * BK) : static_cast<float>(BK);
       const float w = drop ? nj * expf(s - M) : 0.f;
       lacc += w;
       uint32_t dm = __ballot_sync(0xffffffffu, drop);
@@ -305,6 +305,16 @@ __device__ __forceinline__ void route_query_block(SmemCtl<C> &sc, RouteSlot<C> &
   }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) lacc += __shfl_xor_sync(0xffffffffu, lacc, off);
+}
+
+template <class C>
+__device__ __forceinline__ void route_query_block(SmemCtl<C> &sc, RouteSlot<C> &rs, const FwdParams &p,
+                                                  int bh, int sb, int qb, int lane) {
+  constexpr int VPL = C::D / 32;
+  const bool correct = (p.mode == 2);
+  float cacc[VPL];
+  float lacc, M;
+  route_scan<C::D, C::BQ, C::BK>(p, bh, qb, lane, correct, sc.mask[sb], cacc, lacc, M);
 #pragma unroll
   for (int e = 0; e < VPL; ++e) rs.Cv[sb][lane * VPL + e] = correct ? cacc[e] : 0.f;
   if (lane == 0) {
@@ -326,7 +336,10 @@ __device__ void run_router(SmemCtl<C> &sc, const FwdParams &p, int lane) {
     bool w_ok = mbar_wait(&sc.route_empty[s], ((r_it >> 1) & 1) ^ 1, p.timeout_ns, ab);
     if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
     int item = 0;
-    if (lane == 0) item = static_cast<int>(atomicAdd(p.counter, 1u));
+    if (lane == 0) {
+      item = static_cast<int>(atomicAdd(p.counter, 1u));
+      if (p.order && item < p.n_items) item = p.order[item];  // planned order
+    }
     item = __shfl_sync(0xffffffffu, item, 0);
     RouteSlot<C> &rs = sc.route[s];
     if (item >= p.n_items) {
@@ -857,6 +870,101 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
     __syncwarp();
     tc_fence_after_sync();
     tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------------ planning pass
+
+// Work-item schedule for the attention kernel. Each warp routes one item (query tile)
+// exactly as the kernel's router will and records how many key blocks the tile keeps
+// (its cost; nothing else about the keep sets leaves the chip). The last block to finish
+// then orders the items: groups of `group_heads` consecutive heads in head order (the
+// group's K/V stays resident in L2), and within a group the costliest items first, so
+// the short items fill the end of the kernel instead of long ones starting late.
+template <int D, int BQ, int BK, int SUBQ>
+__global__ void __launch_bounds__(256) plan_kernel(const FwdParams p, int *cost, int *order, unsigned int *done,
+                                                   int group_heads) {
+  constexpr int WARPS = 8;
+  __shared__ uint32_t mask[WARPS][SUBQ][kMaskWords];
+  __shared__ int hist[kMaxKeyBlocks + 2];
+  __shared__ int warp_tot[WARPS];
+  __shared__ int is_last;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nW = (p.nKB + 31) >> 5;
+  const int item = blockIdx.x * WARPS + warp;
+  if (item < p.n_items) {
+    const int bh = item / p.items_per_head;
+    const int tile = item - bh * p.items_per_head;
+    for (int sb = 0; sb < SUBQ; ++sb)
+      for (int w = lane; w < nW; w += 32) mask[warp][sb][w] = 0u;
+    __syncwarp();
+    float cacc[D / 32];
+    float lacc, M;
+    for (int sb = 0; sb < SUBQ; ++sb) {
+      const int qb = tile * SUBQ + sb;
+      if (qb < p.nQB) route_scan<D, BQ, BK>(p, bh, qb, lane, false, mask[warp][sb], cacc, lacc, M);
+    }
+    __syncwarp();
+    int cnt = 0;
+    for (int w = lane; w < nW; w += 32) {
+      uint32_t u = 0;
+      for (int sb = 0; sb < SUBQ; ++sb) u |= mask[warp][sb][w];
+      cnt += __popc(u);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, off);
+    if (lane == 0) cost[item] = cnt;
+  }
+  // The last block to finish builds the order.
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) is_last = (atomicAdd(done, 1u) == gridDim.x - 1);
+  __syncthreads();
+  if (!is_last) return;
+  __threadfence();
+  const int BH = p.n_items / p.items_per_head;
+  const int nbins = p.nKB + 1;  // cost in [0, nKB]
+  for (int h0 = 0; h0 < BH; h0 += group_heads) {
+    const int i0 = h0 * p.items_per_head;
+    const int i1 = min(BH, h0 + group_heads) * p.items_per_head;
+    for (int c = threadIdx.x; c < nbins; c += blockDim.x) hist[c] = 0;
+    __syncthreads();
+    for (int i = i0 + threadIdx.x; i < i1; i += blockDim.x) atomicAdd(&hist[cost[i]], 1);
+    __syncthreads();
+    // Exclusive scan over descending cost: start[c] = number of items costlier than c.
+    // Each thread owns a contiguous run of bins (from the costliest end).
+    const int per = (nbins + blockDim.x - 1) / blockDim.x;
+    const int c_hi = nbins - 1 - threadIdx.x * per;  // this thread's bins: c_hi, c_hi-1, ...
+    int local = 0;
+    for (int k = 0; k < per; ++k) {
+      const int c = c_hi - k;
+      if (c >= 0) local += hist[c];
+    }
+    int incl = local;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += y;
+    }
+    if (lane == 31) warp_tot[warp] = incl;
+    __syncthreads();
+    int before = 0;
+    for (int w = 0; w < warp; ++w) before += warp_tot[w];
+    int run = before + incl - local;
+    for (int k = 0; k < per; ++k) {
+      const int c = c_hi - k;
+      if (c >= 0) {
+        const int cnt_c = hist[c];
+        hist[c] = run;
+        run += cnt_c;
+      }
+    }
+    __syncthreads();
+    for (int i = i0 + threadIdx.x; i < i1; i += blockDim.x) {
+      const int pos = atomicAdd(&hist[cost[i]], 1);
+      order[i0 + pos] = i;
+    }
+    __syncthreads();
   }
 }
 

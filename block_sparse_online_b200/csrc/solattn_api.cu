@@ -17,7 +17,7 @@ namespace {
 using namespace solattn;
 
 constexpr size_t kAlign = 256;
-constexpr size_t kHeaderBytes = 256;  // [0]: work counter (u32), [4]: status word (i32)
+constexpr size_t kHeaderBytes = 256;  // [0]: work counter (u32), [4]: status word (i32), [8]: plan counter
 constexpr unsigned long long kDefaultTimeoutNs = 2000000000ull;  // 2 s per device-side wait
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -27,7 +27,7 @@ int nblocks(int N, int blk) { return (N + blk - 1) / blk; }
 bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 struct WsLayout {
-  size_t qbar, kbar, vbar, v16, total;
+  size_t qbar, kbar, vbar, v16, cost, order, total;
 };
 
 int check_shape(int B, int H, int N, int d, int Bq, int Bk) {
@@ -46,7 +46,10 @@ WsLayout ws_layout(int B, int H, int N, int d, int Bq, int Bk) {
   w.kbar = w.qbar + align_up(bh * nblocks(N, Bq) * d * sizeof(float), kAlign);
   w.vbar = w.kbar + align_up(bh * nblocks(N, Bk) * d * sizeof(float), kAlign);
   w.v16 = w.vbar + align_up(bh * nblocks(N, Bk) * d * sizeof(float), kAlign);
-  w.total = w.v16 + align_up(bh * N * d * 2, kAlign);
+  const size_t items = bh * static_cast<size_t>(nblocks(N, 128));  // one work item per 128-row tile
+  w.cost = w.v16 + align_up(bh * N * d * 2, kAlign);
+  w.order = w.cost + align_up(items * sizeof(int), kAlign);
+  w.total = w.order + align_up(items * sizeof(int), kAlign);
   return w;
 }
 
@@ -140,8 +143,29 @@ template <int D, int BK, int SUBQ>
 int dispatch_tiles(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv, FwdParams p, int sms,
                    cudaStream_t st) {
   using C = Cfg<D, BK, SUBQ>;
-  p.items_per_head = (p.N + C::TILE_M - 1) / C::TILE_M;
   return launch_fwd<C>(mq, mk, mv, p, sms, st);
+}
+
+template <int D, int BK, int SUBQ>
+int launch_plan(const FwdParams &p, int *cost, int *order, unsigned int *done, int group_heads, cudaStream_t st) {
+  const int grid = (p.n_items + 7) / 8;
+  plan_kernel<D, 128 / SUBQ, BK, SUBQ><<<grid, 256, 0, st>>>(p, cost, order, done, group_heads);
+  return cudaGetLastError() == cudaSuccess ? SOLATTN_OK : SOLATTN_ECUDA;
+}
+
+int dispatch_plan(int d, int Bq, int Bk, const FwdParams &p, int *cost, int *order, unsigned int *done,
+                  int group_heads, cudaStream_t st) {
+  const int subq = 128 / Bq;
+  if (d == 128) {
+    if (Bk == 128) return subq == 1 ? launch_plan<128, 128, 1>(p, cost, order, done, group_heads, st)
+                                    : launch_plan<128, 128, 2>(p, cost, order, done, group_heads, st);
+    return subq == 1 ? launch_plan<128, 64, 1>(p, cost, order, done, group_heads, st)
+                     : launch_plan<128, 64, 2>(p, cost, order, done, group_heads, st);
+  }
+  if (Bk == 128) return subq == 1 ? launch_plan<64, 128, 1>(p, cost, order, done, group_heads, st)
+                                  : launch_plan<64, 128, 2>(p, cost, order, done, group_heads, st);
+  return subq == 1 ? launch_plan<64, 64, 1>(p, cost, order, done, group_heads, st)
+                   : launch_plan<64, 64, 2>(p, cost, order, done, group_heads, st);
 }
 
 int dispatch(int d, int Bq, int Bk, const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
@@ -258,6 +282,21 @@ int forward_impl(const void *q, const void *k, const void *v, void *out, int B, 
   p.counter = reinterpret_cast<unsigned int *>(ws);
   p.status = reinterpret_cast<int *>(ws + 4);
   p.timeout_ns = kDefaultTimeoutNs;
+  p.items_per_head = nblocks(N, 128);
+  p.order = nullptr;
+  if (mode != SOLATTN_DENSE) {
+    // Schedule: heads in groups whose K and V16 fit in ~64 MB of L2 together, costliest
+    // tiles first within a group.
+    const size_t head_kv = static_cast<size_t>(N) * d * 4;
+    int group_heads = static_cast<int>((64ull << 20) / (head_kv ? head_kv : 1));
+    group_heads = group_heads < 1 ? 1 : (group_heads > BH ? BH : group_heads);
+    int *cost = reinterpret_cast<int *>(ws + wl.cost);
+    int *order = reinterpret_cast<int *>(ws + wl.order);
+    const int rp = dispatch_plan(d, Bq, Bk, p, cost, order, reinterpret_cast<unsigned int *>(ws + 8), group_heads,
+                                 st);
+    if (rp != SOLATTN_OK) return rp;
+    p.order = order;
+  }
   if (ev_attn_begin && cudaEventRecord(static_cast<cudaEvent_t>(ev_attn_begin), st) != cudaSuccess)
     return SOLATTN_ECUDA;
   const int rl = dispatch(d, Bq, Bk, mq, mk, mv, p, di.sms, st);
