@@ -5,8 +5,9 @@
 // the list of key blocks kept by any of the tile's query blocks. Roles, by warp:
 //   warp 0      TMA producer: the item's Q tile (double-buffered across items), then
 //               K_j and V_j of every kept block into a ring of shared-memory slots.
-//   warp 1      MMA issuer (one thread): S = Q K_j^T into tensor memory (TMEM,
-//               bf16 -> fp32), O += P V_j with P read from TMEM (fp16 -> fp32).
+//   warps 1, 3  MMA issuers (one thread each, for warpgroups A and B, taking turns):
+//               S = Q K_j^T into tensor memory (TMEM, bf16 -> fp32), O += P V_j with P
+//               read from TMEM (fp16 -> fp32).
 //   warp 2      router: on-the-fly block thresholding and the correction sums for the
 //               NEXT item (double-buffered), from the fp32 pooled blocks in L2.
 //   warps 4..7  softmax warpgroup A, warps 8..11 softmax warpgroup B. The tile's kept
@@ -14,7 +15,7 @@
 //               5, ...); each keeps its own S, O, running max and sum for all 128 rows.
 //               At the end of the item they exchange max and sum through shared memory
 //               and each writes half of the output columns of the merged result.
-// The MMA warp alternates A and B (ping-pong): while one warpgroup exponentiates its
+// The MMA groups alternate A and B (ping-pong): while one warpgroup exponentiates its
 // S tile, the tensor core runs the other's P V and next Q K^T. Every K/V block is
 // loaded once.
 //
@@ -93,7 +94,7 @@ struct Cfg {
   static constexpr int WG_COLS = BK + D;     // TMEM columns per warpgroup: S (aliased by P) + O
   static constexpr int TMEM_NEED = NWG * WG_COLS;
   static constexpr int TMEM_COLS = TMEM_NEED <= 64 ? 64 : TMEM_NEED <= 128 ? 128 : TMEM_NEED <= 256 ? 256 : 512;
-  // One control warpgroup (warp 0 producer, warp 1 MMA, warp 2 router, warp 3 spare)
+  // One control warpgroup (warp 0 producer, warps 1 and 3 MMA issuers, warp 2 router)
   // and two softmax warpgroups. A warp may only touch TMEM lanes 32*(warp%4)..+31, so
   // each softmax warpgroup covers the four lane quadrants once.
   static constexpr int CTRL_WARPS = 4;
@@ -135,7 +136,8 @@ struct SmemCtl {
   uint64_t s_full[C::NWG], p_full[C::NWG], xchg[C::NWG];
   uint64_t o_full, o_empty;
   uint64_t route_full[2], route_empty[2];
-  uint64_t mma_done;
+  uint64_t mma_done[C::NWG];
+  uint32_t mma_group;  // number of MMA groups issued so far (turn of the two MMA threads)
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -512,13 +514,46 @@ __device__ __forceinline__ void issue_pv(uint32_t tmem, int w, uint32_t v_base, 
   }
 }
 
+// Ring index (within an item) of V_u and of K_u in the producer's order K_0, K_1, then
+// V_u, K_{u+2} for u = 0..n-1: every position before u contributes its V and, while
+// u' + 2 < n, a K. An item fills 2n entries.
+__device__ __forceinline__ int ring_index_v(int u, int n) {
+  return min(n, 2) + u + min(u, max(n - 2, 0));
+}
+__device__ __forceinline__ int ring_index_k(int u, int n) {
+  return u < 2 ? u : ring_index_v(u - 2, n) + 1;
+}
+
+// Wait (bounded) until the shared MMA group counter reaches `target`.
+__device__ __forceinline__ bool wait_turn(const volatile uint32_t *gidx, uint32_t target, uint64_t limit_ns,
+                                          const volatile int *abort_flag) {
+  if (*gidx == target) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (*gidx == target) return true;
+    if ((it & 255u) == 0u) {
+      if (*abort_flag) return false;
+      if (global_timer_ns() - t0 > limit_ns) return false;
+    }
+  }
+}
+
+// MMA issue, one thread per softmax warpgroup w. Thread w issues, for the positions u =
+// w, w + 2, ... of each item's kept list, the group O_w += P_w V_u followed by
+// S_w = Q K_{u+2}^T (and the first S_w of the item up front). The two threads take
+// turns through a shared group counter, so the tensor core sees the groups in the
+// order A, B, A, B, ... while each thread does its barrier waits (K/V landed, P ready)
+// during the other's issue: tcgen05 issue advances only as fast as the tensor core
+// drains, so waits between groups would otherwise leave it idle.
+// Group numbering within an item of n kept blocks: S_A(0) = 0, S_B(1) = 1, step u =
+// 2 + u (for n == 1: S_A(0) = 0, step 0 = 1); an item has n + 2 groups (2 if n == 1).
 template <class C>
-__device__ void run_mma(SmemCtl<C> &sc, const FwdParams &p, uint32_t tmem, uint8_t *q_smem, uint8_t *ring) {
+__device__ void run_mma(SmemCtl<C> &sc, const FwdParams &p, uint32_t tmem, uint8_t *q_smem, uint8_t *ring, int w) {
   const volatile int *ab = &sc.abort_flag;
+  volatile uint32_t *gidx = &sc.mma_group;
   const uint32_t q_base = smem_u32(q_smem);
   const uint32_t ring_base = smem_u32(ring);
-  uint32_t kv_it = 0, q_it = 0, o_it = 0;
-  uint32_t p_ph[C::NWG] = {0, 0};
+  uint32_t kv_base = 0, q_it = 0, o_it = 0, p_ph = 0, g_base = 0;
   bool ok = true;
   auto wait = [&](uint64_t *bar, uint32_t par) {
     if (!ok) return false;
@@ -526,11 +561,17 @@ __device__ void run_mma(SmemCtl<C> &sc, const FwdParams &p, uint32_t tmem, uint8
     else tc_fence_after_sync();
     return ok;
   };
-  // Next ring slot, once its copy has landed (-1 on timeout).
-  auto next_slot = [&]() {
-    const int slot = kv_it % C::NSLOT;
-    if (!wait(&sc.full[slot], (kv_it / C::NSLOT) & 1)) return -1;
-    ++kv_it;
+  auto turn = [&](uint32_t g) {
+    if (!ok) return false;
+    if (!wait_turn(gidx, g_base + g, p.timeout_ns, ab)) ok = false;
+    return ok;
+  };
+  auto pass_turn = [&](uint32_t g) { *gidx = g_base + g + 1; };
+  // Ring slot of entry e of the current item, once its copy has landed (-1 on timeout).
+  auto slot_of = [&](int e) {
+    const uint32_t gg = kv_base + static_cast<uint32_t>(e);
+    const int slot = gg % C::NSLOT;
+    if (!wait(&sc.full[slot], (gg / C::NSLOT) & 1)) return -1;
     return slot;
   };
   for (uint32_t r_it = 0; ok; ++r_it) {
@@ -540,49 +581,65 @@ __device__ void run_mma(SmemCtl<C> &sc, const FwdParams &p, uint32_t tmem, uint8
     const int item = rs.item;
     if (item < 0) break;
     const int n = rs.n_union;
-    const int qb = q_it & 1;
-    if (!wait(&sc.q_full[qb], (q_it >> 1) & 1)) break;
+    const int qb = q_it % C::NQBUF;
+    if (!wait(&sc.q_full[qb], (q_it / C::NQBUF) & 1)) break;
     ++q_it;
     const uint32_t q_addr = q_base + qb * C::Q_TILE_BYTES;
-    // Prologue: S for the first kept block of each warpgroup.
-    for (int u0 = 0; u0 < n && u0 < 2; ++u0) {
-      const int ks = next_slot();
-      if (ks < 0) break;
-      issue_qk<C>(tmem, u0, q_addr, ring_base + ks * C::KV_BYTES);
-      tc_commit(&sc.s_full[u0]);
+    // last position of this warpgroup whose S is issued (-1 if none)
+    const int last_s = (n > w) ? (((n - 1 - w) & ~1) + w) : -1;
+    if (w < n) {
+      const int ks = slot_of(ring_index_k(w, n));
+      if (ks < 0 || !turn(w)) break;
+      issue_qk<C>(tmem, w, q_addr, ring_base + ks * C::KV_BYTES);
+      tc_commit(&sc.s_full[w]);
       tc_commit(&sc.empty[ks]);
+      if (last_s == w) tc_commit(&sc.q_empty[qb]);
+      pass_turn(w);
+    } else {
+      mbar_arrive(&sc.q_empty[qb]);  // no S for this warpgroup in this item
     }
-    if (!ok) break;
-    if (n <= 2) tc_commit(&sc.q_empty[qb]);
-    for (int u = 0; u < n && ok; ++u) {
-      const int w = u & 1;
-      const int vs = next_slot();
+    bool first = true;
+    for (int u = w; u < n && ok; u += 2) {
+      const int vs = slot_of(ring_index_v(u, n));
       if (vs < 0) break;
-      if (!wait(&sc.p_full[w], p_ph[w])) break;
-      p_ph[w] ^= 1;
+      if (!wait(&sc.p_full[w], p_ph)) break;
+      p_ph ^= 1;
       // The first P V of the item overwrites O: the previous item's epilogue must be done.
-      if (u == 0 && !wait(&sc.o_empty, (o_it & 1) ^ 1)) break;
-      issue_pv<C>(tmem, w, ring_base + vs * C::KV_BYTES, u >= 2);
-      tc_commit(&sc.empty[vs]);
+      if (first && !wait(&sc.o_empty, (o_it & 1) ^ 1)) break;
+      int ks = -1;
       if (u + 2 < n) {
-        const int ks = next_slot();
+        ks = slot_of(ring_index_k(u + 2, n));
         if (ks < 0) break;
+      }
+      const uint32_t g = (n == 1) ? 1u : static_cast<uint32_t>(2 + u);
+      if (!turn(g)) break;
+      issue_pv<C>(tmem, w, ring_base + vs * C::KV_BYTES, !first);
+      first = false;
+      tc_commit(&sc.empty[vs]);
+      if (ks >= 0) {
         issue_qk<C>(tmem, w, q_addr, ring_base + ks * C::KV_BYTES);
         tc_commit(&sc.s_full[w]);
         tc_commit(&sc.empty[ks]);
-        if (u + 2 == n - 1) tc_commit(&sc.q_empty[qb]);
+        if (u + 2 == last_s) tc_commit(&sc.q_empty[qb]);
       }
+      pass_turn(g);
     }
     if (!ok) break;
-    tc_commit(&sc.o_full);
+    if (first) {  // no P V for this warpgroup in this item (n == 1, w == 1)
+      mbar_arrive(&sc.o_full);
+    } else {
+      tc_commit(&sc.o_full);
+    }
     ++o_it;
+    kv_base += 2 * static_cast<uint32_t>(n);
+    g_base += (n == 1) ? 2u : static_cast<uint32_t>(n + 2);
     mbar_arrive(&sc.route_empty[s]);
   }
   if (!ok) raise_abort(&sc.abort_flag, p.status);
   // Every tcgen05 operation issued here must finish before TMEM is released.
   const int zero = 0;
-  tc_commit(&sc.mma_done);
-  mbar_wait(&sc.mma_done, 0, p.timeout_ns, &zero);
+  tc_commit(&sc.mma_done[w]);
+  mbar_wait(&sc.mma_done[w], 0, p.timeout_ns, &zero);
 }
 
 // ------------------------------------------------------------------ softmax / epilogue
@@ -819,20 +876,21 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
     }
     for (int i = 0; i < C::NQBUF; ++i) {
       mbar_init(&sc.q_full[i], 1);
-      mbar_init(&sc.q_empty[i], 1);
+      mbar_init(&sc.q_empty[i], C::NWG);  // released by both MMA threads
     }
     for (int w = 0; w < C::NWG; ++w) {
       mbar_init(&sc.s_full[w], 1);
       mbar_init(&sc.p_full[w], 128);
       mbar_init(&sc.xchg[w], 128);
     }
-    mbar_init(&sc.o_full, 1);
+    mbar_init(&sc.o_full, C::NWG);  // one commit (or arrive) per MMA thread
     mbar_init(&sc.o_empty, 128 * C::NWG);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&sc.route_full[s], 1);
-      mbar_init(&sc.route_empty[s], 2 + 128 * C::NWG);
+      mbar_init(&sc.route_empty[s], 1 + C::NWG + 128 * C::NWG);  // producer, MMA threads, softmax
     }
-    mbar_init(&sc.mma_done, 1);
+    for (int w = 0; w < C::NWG; ++w) mbar_init(&sc.mma_done[w], 1);
+    sc.mma_group = 0;
     sc.abort_flag = 0;
     fence_mbar_init();
   }
@@ -854,8 +912,8 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
     regs_dec<C::CTRL_REGS>();
     if (warp == 0) {
       if (lane == 0) run_producer<C>(sc, p, q_smem, ring, &tm_q, &tm_k, &tm_v);
-    } else if (warp == 1) {
-      if (lane == 0) run_mma<C>(sc, p, tmem, q_smem, ring);
+    } else if (warp == 1 || warp == 3) {
+      if (lane == 0) run_mma<C>(sc, p, tmem, q_smem, ring, warp == 1 ? 0 : 1);
     } else if (warp == 2) {
       run_router<C>(sc, p, lane);
     }
