@@ -101,8 +101,10 @@ struct Cfg {
   static constexpr int NUM_THREADS = 32 * CTRL_WARPS + 128 * NWG;
   // Register split: the control warpgroup hands registers to the softmax warpgroups.
   // The sum stays within the registers the block is launched with (384 threads x 168).
-  static constexpr int CTRL_REGS = 120;
-  static constexpr int SOFTMAX_REGS = 192;
+  // The softmax streams S in 32-column chunks (about 100 live registers); the router and
+  // MMA issuers spill below about 150.
+  static constexpr int CTRL_REGS = 152;
+  static constexpr int SOFTMAX_REGS = 176;
   static_assert(128 * CTRL_REGS + 256 * SOFTMAX_REGS <= 384 * 168, "register split");
   // S = Q K^T in bf16; O += P V in fp16 (P in [0, 2^8] after the lazy rescale; V is the
   // fp16 copy written by the pooling pass).
@@ -491,32 +493,30 @@ __device__ void run_producer(SmemCtl<C> &sc, const FwdParams &p, uint8_t *q_smem
 
 // ------------------------------------------------------------------ MMA issuer
 
+// MMA issue takes prebuilt shared-memory descriptors of the operand tiles and adds only
+// compile-time offsets per 16-wide k step (the start-address field counts 16-byte units
+// and never carries, as shared memory ends below 256 KB): building descriptors per
+// instruction starves the tensor core when the softmax warps keep the issue slots busy.
 template <class C>
-__device__ __forceinline__ void issue_qk(uint32_t tmem, int w, uint32_t q_base, uint32_t k_base) {
+__device__ __forceinline__ void issue_qk(uint32_t tmem, int w, uint64_t q_desc, uint64_t k_desc) {
   const uint32_t d_tmem = tmem + w * C::WG_COLS;
 #pragma unroll
   for (int kk = 0; kk < C::D / 16; ++kk) {
-    const uint32_t off_q = (kk >> 2) * (C::TILE_M * 128) + (kk & 3) * 32;
-    const uint32_t off_k = (kk >> 2) * (C::BK * 128) + (kk & 3) * 32;
-    mma_bf16_ss(d_tmem, smem_desc_sw128(q_base + off_q, 16, 1024), smem_desc_sw128(k_base + off_k, 16, 1024),
-                C::IDESC_QK, kk > 0 ? 1u : 0u);
+    const uint64_t off_q = static_cast<uint64_t>((kk >> 2) * (C::TILE_M * 128 / 16) + (kk & 3) * 2);
+    const uint64_t off_k = static_cast<uint64_t>((kk >> 2) * (C::BK * 128 / 16) + (kk & 3) * 2);
+    mma_bf16_ss(d_tmem, q_desc + off_q, k_desc + off_k, C::IDESC_QK, kk > 0 ? 1u : 0u);
   }
 }
-
 template <class C>
-__device__ __forceinline__ void issue_pv(uint32_t tmem, int w, uint32_t v_base, bool accumulate) {
+__device__ __forceinline__ void issue_pv(uint32_t tmem, int w, uint64_t v_desc, bool accumulate) {
   const uint32_t d_tmem = tmem + w * C::WG_COLS + C::BK;
   const uint32_t p_tmem = tmem + w * C::WG_COLS;
 #pragma unroll
   for (int kk = 0; kk < C::BK / 16; ++kk) {
-    mma_bf16_ts(d_tmem, p_tmem + kk * 8, smem_desc_sw128(v_base + kk * (16 * 128), C::BK * 128, 1024),
-                C::IDESC_PV, (accumulate || kk > 0) ? 1u : 0u);
+    mma_bf16_ts(d_tmem, p_tmem + kk * 8, v_desc + static_cast<uint64_t>(kk * (16 * 128 / 16)), C::IDESC_PV,
+                (accumulate || kk > 0) ? 1u : 0u);
   }
 }
-
-// Ring index (within an item) of V_u and of K_u in the producer's order K_0, K_1, then
-// V_u, K_{u+2} for u = 0..n-1: every position before u contributes its V and, while
-// u' + 2 < n, a K. An item fills 2n entries.
 __device__ __forceinline__ int ring_index_v(int u, int n) {
   return min(n, 2) + u + min(u, max(n - 2, 0));
 }
@@ -551,8 +551,12 @@ template <class C>
 __device__ void run_mma(SmemCtl<C> &sc, const FwdParams &p, uint32_t tmem, uint8_t *q_smem, uint8_t *ring, int w) {
   const volatile int *ab = &sc.abort_flag;
   volatile uint32_t *gidx = &sc.mma_group;
-  const uint32_t q_base = smem_u32(q_smem);
-  const uint32_t ring_base = smem_u32(ring);
+  // Descriptors of Q buffer 0 and of ring slot 0 (as a K tile and as a V tile); other
+  // buffers and slots are whole multiples of 16 bytes further on.
+  const uint64_t q_desc0 = smem_desc_sw128(smem_u32(q_smem), 16, 1024);
+  const uint64_t k_desc0 = smem_desc_sw128(smem_u32(ring), 16, 1024);
+  const uint64_t v_desc0 = smem_desc_sw128(smem_u32(ring), C::BK * 128, 1024);
+  constexpr uint32_t kSlotUnits = C::KV_BYTES / 16;
   uint32_t kv_base = 0, q_it = 0, o_it = 0, p_ph = 0, g_base = 0;
   bool ok = true;
   auto wait = [&](uint64_t *bar, uint32_t par) {
@@ -584,16 +588,12 @@ __device__ void run_mma(SmemCtl<C> &sc, const FwdParams &p, uint32_t tmem, uint8
     const int qb = q_it % C::NQBUF;
     if (!wait(&sc.q_full[qb], (q_it / C::NQBUF) & 1)) break;
     ++q_it;
-    const uint32_t q_addr = q_base + qb * C::Q_TILE_BYTES;
-    // last position of this warpgroup whose S is issued (-1 if none)
-    const int last_s = (n > w) ? (((n - 1 - w) & ~1) + w) : -1;
+    const uint64_t q_desc = q_desc0 + static_cast<uint64_t>(qb * (C::Q_TILE_BYTES / 16));
     if (w < n) {
       const int ks = slot_of(ring_index_k(w, n));
       if (ks < 0 || !turn(w)) break;
-      issue_qk<C>(tmem, w, q_addr, ring_base + ks * C::KV_BYTES);
+      issue_qk<C>(tmem, w, q_desc, k_desc0 + static_cast<uint64_t>(ks * kSlotUnits));
       tc_commit(&sc.s_full[w]);
-      tc_commit(&sc.empty[ks]);
-      if (last_s == w) tc_commit(&sc.q_empty[qb]);
       pass_turn(w);
     } else {
       mbar_arrive(&sc.q_empty[qb]);  // no S for this warpgroup in this item
@@ -613,14 +613,11 @@ __device__ void run_mma(SmemCtl<C> &sc, const FwdParams &p, uint32_t tmem, uint8
       }
       const uint32_t g = (n == 1) ? 1u : static_cast<uint32_t>(2 + u);
       if (!turn(g)) break;
-      issue_pv<C>(tmem, w, ring_base + vs * C::KV_BYTES, !first);
+      issue_pv<C>(tmem, w, v_desc0 + static_cast<uint64_t>(vs * kSlotUnits), !first);
       first = false;
-      tc_commit(&sc.empty[vs]);
       if (ks >= 0) {
-        issue_qk<C>(tmem, w, q_addr, ring_base + ks * C::KV_BYTES);
+        issue_qk<C>(tmem, w, q_desc, k_desc0 + static_cast<uint64_t>(ks * kSlotUnits));
         tc_commit(&sc.s_full[w]);
-        tc_commit(&sc.empty[ks]);
-        if (u + 2 == last_s) tc_commit(&sc.q_empty[qb]);
       }
       pass_turn(g);
     }
@@ -658,6 +655,11 @@ __device__ void run_softmax(SmemCtl<C> &sc, const FwdParams &p, uint32_t tmem, i
   const int sb = (C::SUBQ == 2 ? (row >> 6) : 0);
   const uint32_t row_bit = 1u << sb;
   uint32_t s_ph = 0;
+  uint32_t kv_base = 0;  // ring entries of earlier items (2 per kept block)
+  // One thread per warpgroup returns the ring slots (and the Q buffer) the tensor core
+  // has finished reading: the MMA issuers commit only the barrier this warpgroup waits on.
+  const bool leader = (threadIdx.x & 127) == 0;
+  auto release = [&](int entry) { mbar_arrive(&sc.empty[(kv_base + static_cast<uint32_t>(entry)) % C::NSLOT]); };
   bool ok = true;
   auto wait = [&](uint64_t *bar, uint32_t par) {
     bool wt = mbar_wait(bar, par, p.timeout_ns, ab);
@@ -683,74 +685,76 @@ __device__ void run_softmax(SmemCtl<C> &sc, const FwdParams &p, uint32_t tmem, i
       const int j = rs.jlist[u];
       if (!wait(&sc.s_full[w], s_ph)) break;
       s_ph ^= 1;
-      // S streams through registers 64 columns (two 32-column loads, one wait) at a time
-      // and each 64-column half of P is stored to TMEM as soon as it is packed (fp16
-      // pairs). The reference max only moves when a half exceeds it by more than the
-      // slack; a half of P already stored is then rescaled in TMEM (rare).
-      const bool rk = (mem & row_bit) != 0;
+      // The group that produced this S (O += P V of position u - 2, then S of position u)
+      // is complete: its K and V tiles and, after this warpgroup's last S, Q are free.
+      if (leader) {
+        release(ring_index_k(u, n));
+        if (u >= w + 2) release(ring_index_v(u - 2, n));
+        if (u + 2 >= n) mbar_arrive(&sc.q_empty[r_it % C::NQBUF]);
+      }
+      // Two passes over the row of S, 32 columns per TMEM load, each load issued one chunk
+      // ahead: the row maximum (a tree of three-input max instructions per chunk), then the
+      // exponentials, whose fp16 pairs go back to TMEM 16 columns at a time. The reference
+      // max only moves when the row maximum exceeds it by more than the slack (O and l are
+      // then rescaled once, below).
+      constexpr int NCH = BK / 32;
+      const bool rk = (mem & row_bit) != 0;  // warp-uniform (a warp's rows share a query block)
       const int ncol = (j == p.nKB - 1) ? (p.N - j * BK) : BK;
-      const bool full = rk && ncol == BK;  // warp-uniform: no column of this block masked
-      float alpha = 1.f;  // total rescale of this row's O and l for this S tile
-      float lsum = 0.f;
-#pragma unroll
-      for (int c2 = 0; c2 < BK / 64; ++c2) {
-        uint32_t sr[2][32];
-        tmem_ld32(s_addr + c2 * 64, sr[0]);
-        tmem_ld32(s_addr + c2 * 64 + 32, sr[1]);
+      const bool full = rk && ncol == BK;    // no column of this block masked
+      float mx = -CUDART_INF_F;
+      uint32_t x[32];
+      if (rk) {
+        tmem_ld32(s_addr, x);
         tmem_wait_ld();
-        reg_fence32(sr[0]);
-        reg_fence32(sr[1]);
-        float mx = -CUDART_INF_F;
-        if (full) {
-          mx = fmax3(u2f(sr[0][0]), u2f(sr[0][1]), u2f(sr[0][2]));
+        reg_fence32(x);
 #pragma unroll
-          for (int e = 3; e < 63; e += 2) mx = fmax3(mx, u2f(sr[e >> 5][e & 31]), u2f(sr[(e + 1) >> 5][(e + 1) & 31]));
-          mx = fmaxf(mx, u2f(sr[1][31]));
-        } else if (rk) {
+        for (int c = 0; c < NCH; ++c) {
+          uint32_t y[32];
+          // the next chunk, or (after the last) chunk 0 again for the exponential pass; the
+          // fence keeps the arithmetic on this chunk after the load is issued
+          tmem_ld32(s_addr + ((c + 1) % NCH) * 32, y);
+          reg_fence32(x);
+          float m;
+          if (full) {
+            m = max_tree_bits<32>(x);
+          } else {
+            m = -CUDART_INF_F;
 #pragma unroll
-          for (int e = 0; e < 64; ++e)
-            if (c2 * 64 + e < ncol) mx = fmaxf(mx, u2f(sr[e >> 5][e & 31]));
-        }
-        const float mxs = mx * sc_log2;
-        float a = 1.f;
-        if (mxs > m_ref + kRescaleSlack) {
-          if (m_ref != -CUDART_INF_F) a = ex2_approx(m_ref - mxs);
-          m_ref = mxs;
-        }
-        alpha *= a;
-        lsum *= a;
-        if (c2 > 0 && __any_sync(0xffffffffu, a != 1.f)) {
-          // Rescale the halves of P already in TMEM (their stores must land first).
-          tmem_wait_st();
-          const __half2 a2 = __float2half2_rn(a);
-#pragma unroll 1
-          for (int h = 0; h < c2; ++h) {
-            uint32_t pp[32];
-            tmem_ld32(s_addr + h * 32, pp);
-            tmem_wait_ld();
-            reg_fence32(pp);
-#pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              __half2 v2 = *reinterpret_cast<__half2 *>(&pp[e]);
-              v2 = __hmul2(v2, a2);
-              pp[e] = *reinterpret_cast<uint32_t *>(&v2);
-            }
-            tmem_st32(s_addr + h * 32, pp);
+            for (int e = 0; e < 32; ++e)
+              if (c * 32 + e < ncol) m = fmaxf(m, u2f(x[e]));
           }
-        }
-        const float neg_m = (m_ref == -CUDART_INF_F) ? 0.f : -m_ref;
-        uint32_t pk[32];
-        if (full) {
-          // Packed fp32 pairs; one pair in kPolyEvery goes through the FMA-pipe exp2.
-          const uint64_t scp = f2(sc_log2, sc_log2);
-          const uint64_t nmp = f2(neg_m, neg_m);
-          uint64_t acc = f2(0.f, 0.f);
+          mx = fmaxf(mx, m);
+          asm volatile("" ::"f"(mx));  // the tree stays ahead of the wait
+          tmem_wait_ld();
+          reg_fence32(y);
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const uint64_t x = fma2(f2(u2f(sr[(2 * e) >> 5][(2 * e) & 31]), u2f(sr[(2 * e + 1) >> 5][(2 * e + 1) & 31])),
-                                    scp, nmp);
+          for (int e = 0; e < 32; ++e) x[e] = y[e];
+        }
+      }
+      const float mxs = mx * sc_log2;
+      float alpha = 1.f;  // rescale of this row's O and l for this S tile
+      if (mxs > m_ref + kRescaleSlack) {
+        if (m_ref != -CUDART_INF_F) alpha = ex2_approx(m_ref - mxs);
+        m_ref = mxs;
+      }
+      const float neg_m = (m_ref == -CUDART_INF_F) ? 0.f : -m_ref;
+      float lsum = 0.f;
+      if (full) {
+        // Packed fp32 pairs; one pair in kPolyEvery goes through the FMA-pipe exp2.
+        const uint64_t scp = f2(sc_log2, sc_log2);
+        const uint64_t nmp = f2(neg_m, neg_m);
+        uint64_t acc = f2(0.f, 0.f);
+#pragma unroll
+        for (int c = 0; c < NCH; ++c) {
+          uint32_t y[32];
+          if (c + 1 < NCH) tmem_ld32(s_addr + (c + 1) * 32, y);
+          reg_fence32(x);
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const uint64_t xx = fma2(f2(u2f(x[2 * e]), u2f(x[2 * e + 1])), scp, nmp);
             float x0, x1, p0, p1;
-            f2_split(x, x0, x1);
+            f2_split(xx, x0, x1);
             if ((e % kPolyEvery) == kPolyEvery - 1) {
               exp2_poly_x2(x0, x1, p0, p1);
             } else {
@@ -760,22 +764,39 @@ __device__ void run_softmax(SmemCtl<C> &sc, const FwdParams &p, uint32_t tmem, i
             acc = add2(acc, f2(p0, p1));
             pk[e] = pack_f16x2(p0, p1);
           }
-          float s0, s1;
-          f2_split(acc, s0, s1);
-          lsum += s0 + s1;
-        } else {
+          tmem_st16(s_addr + c * 16, pk);
+          if (c + 1 < NCH) {
+            tmem_wait_ld();
+            reg_fence32(y);
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int col = c2 * 64 + 2 * e;
-            const float x0 = u2f(sr[(2 * e) >> 5][(2 * e) & 31]);
-            const float x1 = u2f(sr[(2 * e + 1) >> 5][(2 * e + 1) & 31]);
-            const float p0 = (rk && col < ncol) ? ex2_approx(fmaf(x0, sc_log2, neg_m)) : 0.f;
-            const float p1 = (rk && col + 1 < ncol) ? ex2_approx(fmaf(x1, sc_log2, neg_m)) : 0.f;
+            for (int e = 0; e < 32; ++e) x[e] = y[e];
+          }
+        }
+        float s0, s1;
+        f2_split(acc, s0, s1);
+        lsum = s0 + s1;
+      } else {
+#pragma unroll
+        for (int c = 0; c < NCH; ++c) {
+          uint32_t y[32];
+          if (rk && c + 1 < NCH) tmem_ld32(s_addr + (c + 1) * 32, y);
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int col = c * 32 + 2 * e;
+            const float p0 = (rk && col < ncol) ? ex2_approx(fmaf(u2f(x[2 * e]), sc_log2, neg_m)) : 0.f;
+            const float p1 = (rk && col + 1 < ncol) ? ex2_approx(fmaf(u2f(x[2 * e + 1]), sc_log2, neg_m)) : 0.f;
             lsum += p0 + p1;
             pk[e] = pack_f16x2(p0, p1);
           }
+          tmem_st16(s_addr + c * 16, pk);
+          if (rk && c + 1 < NCH) {
+            tmem_wait_ld();
+            reg_fence32(y);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) x[e] = y[e];
+          }
         }
-        tmem_st32(s_addr + c2 * 32, pk);
       }
       l = l * alpha + lsum;
       if (__any_sync(0xffffffffu, alpha != 1.f)) {
@@ -800,6 +821,8 @@ __device__ void run_softmax(SmemCtl<C> &sc, const FwdParams &p, uint32_t tmem, i
     // Epilogue: wait for the last P V of both warpgroups, exchange the row max and sum,
     // and write this warpgroup's half of the output columns of the merged rows.
     if (!wait(&sc.o_full, r_it & 1)) break;
+    if (leader && w < n) release(ring_index_v(w + ((n - 1 - w) & ~1), n));  // V of the last P V
+    kv_base += 2 * static_cast<uint32_t>(n);
     sc.xm[w][row] = m_ref;
     sc.xl[w][row] = l;
     mbar_arrive(&sc.xchg[w]);
@@ -876,7 +899,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
     }
     for (int i = 0; i < C::NQBUF; ++i) {
       mbar_init(&sc.q_full[i], 1);
-      mbar_init(&sc.q_empty[i], C::NWG);  // released by both MMA threads
+      mbar_init(&sc.q_empty[i], C::NWG);  // one arrival per softmax warpgroup (or its MMA thread)
     }
     for (int w = 0; w < C::NWG; ++w) {
       mbar_init(&sc.s_full[w], 1);

@@ -196,6 +196,14 @@ __device__ __forceinline__ void reg_fence16(uint32_t (&r)[16]) {
   for (int i = 0; i < 16; ++i) asm volatile("" : "+r"(r[i]));
 }
 
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
@@ -248,6 +256,33 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
+}
+
+// Maximum of W values as a tree of three-input max instructions: depth log3(W) instead
+// of a dependent chain of W/2 (indices are compile-time after unrolling).
+template <int W>
+__device__ __forceinline__ float max_tree(const float (&in)[W]) {
+  if constexpr (W == 1) {
+    return in[0];
+  } else {
+    constexpr int O = (W + 2) / 3;
+    float out[O];
+#pragma unroll
+    for (int i = 0; i < O; ++i)
+      out[i] = fmax3(in[3 * i], in[3 * i + 1 < W ? 3 * i + 1 : W - 1], in[3 * i + 2 < W ? 3 * i + 2 : W - 1]);
+    return max_tree<O>(out);
+  }
+}
+// Same, for values held as raw fp32 bits (as tcgen05.ld returns them).
+template <int W>
+__device__ __forceinline__ float max_tree_bits(const uint32_t (&in)[W]) {
+  constexpr int O = (W + 2) / 3;
+  float out[O];
+#pragma unroll
+  for (int i = 0; i < O; ++i)
+    out[i] = fmax3(__uint_as_float(in[3 * i]), __uint_as_float(in[3 * i + 1 < W ? 3 * i + 1 : W - 1]),
+                   __uint_as_float(in[3 * i + 2 < W ? 3 * i + 2 : W - 1]));
+  return max_tree<O>(out);
 }
 
 __device__ __forceinline__ uint64_t f2(float lo, float hi) {
