@@ -440,7 +440,9 @@ def main():
                          "traffic": None if trec is None else trec["dram_bytes_per_launch"],
                          "kernel": "solattn_fwd_kernel (executed FLOPs per launch / CUDA-event duration)"},
             "e2e": e2e,
-            "gpu_launches": args.steps * (1 if args.mode == "dense" else 2),
+            # per step: pool_kernel (block means and the fp16 copy of V; the copy alone in
+            # dense mode), plan_kernel (keep modes) and solattn_fwd_kernel
+            "gpu_launches": args.steps * (2 if args.mode == "dense" else 3),
             "clocks": clk,
             "cpu_baseline": cpu,
             "sweep": sweep,
