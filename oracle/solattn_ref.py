@@ -22,9 +22,9 @@ n_i = |R_i|; key blocks j with columns C_j, n_j = |C_j|; d = head dim):
    Methodology, "On-the-fly sparsification"; abstract "comparing block proxy
    scores against a threshold during online softmax"): M(t) is the running
    maximum of the proxies visited so far including the current one, and the
-   visited block is kept iff s >= M(t) - tau. The pages' own threshold is a
-   query-dependent mean + beta * std; the running-max form is the reading
-   fixed for this build.
+   visited block is kept iff s >= M(t) - tau. The pages' own threshold, a
+   query-dependent mean + beta * std from pooled-key moments, is implemented
+   beside it (``keep_sets_gaussian``, below).
 5. Output, closed form (no online recurrence):
    keep_correct: O_r = [sum_{j kept} sum_{c in C_j} e^{s_rc} v_c
                         + sum_{j dropped} n_j e^{s_ij} v_j]
@@ -243,6 +243,86 @@ def forward(q, k, v, Bq: int, Bk: int, tau: float, mode="keep_correct", order: s
             pseudo = correction_terms(sbar[b, h, i], ~keep[b, h, i], counts, vbar[b, h])
         out[b, h, rows] = attend_block(q[b, h, rows], k[b, h], v[b, h], kept_cols, pseudo)
     return out, keep
+
+
+# ----------------------------------------------------------------- query-dependent Gaussian threshold
+#
+# The pages' own routing rule (paperlayer summary "Sol-Attn: Accelerating Video
+# Generation Inference via On-the-Fly Attention Sparsification", §2 Block-Sparse
+# Attention, Figure 2: a threshold from the proxy-logit mean mu, standard deviation
+# sigma and a standardized offset beta; §3 Methodology, "Dynamic threshold routing":
+# query-dependent thresholds from proxy-score statistics with one shared standardized
+# cutoff, the mean and variance taken from the pooled keys' first and second moments;
+# App. "Threshold variance derivation" and "Diagonal threshold estimator": the exact
+# variance from the pooled-key covariance, or its diagonal v_K = diag(Cov[K]) only).
+# Readings (the pages do not fix them): the moments run over the key blocks with equal
+# weight and 1/nKB normalisation; a block is kept iff its proxy is >= the threshold;
+# the row's top block (largest proxy, lowest index on ties) is always kept, so no
+# query block's exact set is empty.
+
+def key_moments(kbar: np.ndarray):
+    """Mean and covariance of the pooled keys over the key blocks:
+    [..., nKB, d] -> (mean [..., d], cov [..., d, d]), normalised by 1/nKB."""
+    m = kbar.mean(axis=-2)
+    c = kbar - m[..., None, :]
+    return m, np.swapaxes(c, -1, -2) @ c / kbar.shape[-2]
+
+
+def threshold_variance(qbar: np.ndarray, cov: np.ndarray, variant: str) -> np.ndarray:
+    """sigma_i^2 of the proxies of query block i: q_i^T Cov[K] q_i / d ("exact") or
+    sum_e q_ie^2 Cov[K]_ee / d ("diag"): [..., nQB, d], [..., d, d] -> [..., nQB]."""
+    d = qbar.shape[-1]
+    if variant == "exact":
+        return np.einsum("...id,...de,...ie->...i", qbar, cov, qbar) / d
+    if variant == "diag":
+        return np.einsum("...id,...d->...i", qbar * qbar, np.diagonal(cov, axis1=-2, axis2=-1)) / d
+    raise ValueError(variant)
+
+
+def gaussian_threshold(qbar: np.ndarray, kbar: np.ndarray, beta: float, variant: str = "exact") -> np.ndarray:
+    """theta_i = mu_i + beta * sigma_i with mu_i = q_i . E[K] / sqrt(d): [..., nQB]."""
+    d = qbar.shape[-1]
+    m, cov = key_moments(kbar)
+    mu = np.einsum("...id,...d->...i", qbar, m) / math.sqrt(d)
+    sigma = np.sqrt(np.maximum(threshold_variance(qbar, cov, variant), 0.0))
+    return mu + beta * sigma
+
+
+def gaussian_keep(sbar: np.ndarray, theta: np.ndarray) -> np.ndarray:
+    """Keep iff s_ij >= theta_i, plus the row's top block: [..., nQB, nKB] bool."""
+    keep = sbar >= theta[..., None]
+    top = np.argmax(sbar, axis=-1)
+    np.put_along_axis(keep, top[..., None], True, axis=-1)
+    return keep
+
+
+def keep_sets_gaussian(q, k, Bq: int, Bk: int, beta: float, variant: str = "exact", mode="keep_correct"):
+    """Keep sets under the Gaussian threshold.
+
+    Returns (keep, margin = s - theta (+inf for a top block kept only because it is
+    the top block), sbar), all [B, H, nQB, nKB]. In dense mode, or for beta = -inf,
+    every block is kept.
+    """
+    mode = _mode_name(mode)
+    q, k = as_f64(q), as_f64(k)
+    N = q.shape[-2]
+    qbar, kbar = pool(q, Bq), pool(k, Bk)
+    sbar = proxy(qbar, kbar)
+    if mode == "dense" or beta == -math.inf:
+        return np.ones(sbar.shape, dtype=bool), np.full(sbar.shape, np.inf), sbar
+    theta = gaussian_threshold(qbar, kbar, beta, variant)
+    keep = gaussian_keep(sbar, theta)
+    margin = sbar - theta[..., None]
+    margin = np.where(keep & (margin < 0), np.inf, margin)
+    return keep, margin, sbar
+
+
+def forward_gaussian(q, k, v, Bq: int, Bk: int, beta: float, variant: str = "exact", mode="keep_correct",
+                     keep: np.ndarray | None = None, qblocks=None):
+    """Output under the Gaussian threshold (steps 1, 2 and 5 as in ``forward``)."""
+    if keep is None:
+        keep, _, _ = keep_sets_gaussian(q, k, Bq, Bk, beta, variant, mode)
+    return forward(q, k, v, Bq, Bk, 0.0, mode, keep=keep, qblocks=qblocks)
 
 
 def sample_qblocks(B, H, nQB, Bq, Bk, nKB, per_head=64, seed=0):

@@ -253,6 +253,83 @@ PINS = [pin_handworked, pin_pool_is_block_mean, pin_dense_is_softmax_attention,
         pin_brute_force_tiny]
 
 
+# ------------------------------------------------- query-dependent Gaussian threshold
+
+def _block_constant_keys(kbar_rows, blk):
+    """K whose blocks of blk tokens are constant rows (so the pooled keys are those rows)."""
+    return np.repeat(kbar_rows, blk, axis=-2)
+
+
+def pin_gaussian_matches_row_statistics():
+    # The exact variant's mu_i and sigma_i are the mean and (1/nKB) standard deviation of
+    # query block i's proxy row, whatever the keys: computed here from the row directly.
+    q, k, _ = _rand(1, 2, 1000, 32, seed=21, scale=1.3)
+    sbar = ref.proxy(ref.pool(q, 64), ref.pool(k, 64))
+    for beta in (-0.7, 0.0, 1.0, 2.5):
+        theta = ref.gaussian_threshold(ref.pool(q, 64), ref.pool(k, 64), beta, "exact")
+        want = sbar.mean(axis=-1) + beta * sbar.std(axis=-1)
+        np.testing.assert_allclose(theta, want, rtol=1e-11, atol=1e-11)
+
+
+def pin_gaussian_diagonal_design():
+    # Pooled keys k_j = a * h_j with h_j the rows of columns 1..d of a 2d x 2d Sylvester
+    # Hadamard matrix: the columns are orthogonal and zero-mean, so the mean is 0 and
+    # Cov[K] = diag(a^2) exactly. Then sigma_i^2 = sum_e q_ie^2 a_e^2 / d for both variants.
+    d, blk = 16, 4
+    H = np.array([[1.0]])
+    while H.shape[0] < 2 * d:
+        H = np.block([[H, H], [H, -H]])
+    rng = np.random.default_rng(5)
+    a = rng.uniform(0.5, 2.0, d)
+    krows = H[:, 1:d + 1] * a  # [2d, d]
+    k = _block_constant_keys(krows, blk)[None, None]
+    q = rng.standard_normal((1, 1, k.shape[2], d))
+    qbar = ref.pool(q, blk)
+    want = np.sqrt((qbar ** 2 * a ** 2).sum(axis=-1) / d)
+    for variant in ("exact", "diag"):
+        theta = ref.gaussian_threshold(qbar, ref.pool(k, blk), 1.0, variant)
+        np.testing.assert_allclose(theta, want, rtol=1e-12, atol=1e-12)
+
+
+def pin_gaussian_keep_fraction():
+    # i.i.d. Gaussian pooled keys: each proxy row is (close to) normal with the row's own
+    # mean and std, so the kept fraction approaches 1 - Phi(beta).
+    d, blk, nkb = 32, 2, 2048
+    rng = np.random.default_rng(8)
+    k = _block_constant_keys(rng.standard_normal((nkb, d)), blk)[None, None]
+    q = rng.standard_normal((1, 1, 64 * blk, d)) + 0.3
+    for beta, frac in ((0.0, 0.5), (1.0, 0.158655), (2.0, 0.022750)):
+        keep, _, _ = ref.keep_sets_gaussian(q, k, blk, blk, beta, "exact")
+        assert abs(keep.mean() - frac) < 0.02 + 0.1 * frac, (beta, keep.mean())
+
+
+def pin_gaussian_limits_and_monotone():
+    q, k, _ = _rand(1, 2, 777, 16, seed=4)
+    sbar = ref.proxy(ref.pool(q, 64), ref.pool(k, 64))
+    keep, _, _ = ref.keep_sets_gaussian(q, k, 64, 64, -math.inf, "exact")
+    assert keep.all()
+    keep, _, _ = ref.keep_sets_gaussian(q, k, 64, 64, 1e9, "diag")
+    assert (keep.sum(axis=-1) == 1).all()
+    assert (np.argmax(keep, axis=-1) == np.argmax(sbar, axis=-1)).all()
+    prev = None
+    for beta in (-1.0, 0.0, 0.5, 1.0, 2.0):
+        cur, _, _ = ref.keep_sets_gaussian(q, k, 64, 64, beta, "exact")
+        assert (cur.sum(axis=-1) >= 1).all()
+        if prev is not None:
+            assert not (cur & ~prev).any()  # a larger beta keeps a subset
+        prev = cur
+    # correlated keys: the diagonal estimator differs from the exact one
+    kc = k.copy()
+    kc[..., 1] = kc[..., 0] * 0.9 + 0.1 * kc[..., 1]
+    t_ex = ref.gaussian_threshold(ref.pool(q, 64), ref.pool(kc, 64), 1.0, "exact")
+    t_dg = ref.gaussian_threshold(ref.pool(q, 64), ref.pool(kc, 64), 1.0, "diag")
+    assert np.abs(t_ex - t_dg).max() > 1e-3
+
+
+PINS += [pin_gaussian_matches_row_statistics, pin_gaussian_diagonal_design, pin_gaussian_keep_fraction,
+         pin_gaussian_limits_and_monotone]
+
+
 @pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
 def test_pin(pin):
     pin()
@@ -313,6 +390,31 @@ def _mut_attend_scale_d(q_rows, k, v, kept_cols, pseudo):
                                         kept_cols, pseudo)
 
 
+def _mut_moments_sample(kbar):
+    m = kbar.mean(axis=-2)
+    c = kbar - m[..., None, :]
+    return m, np.swapaxes(c, -1, -2) @ c / (kbar.shape[-2] - 1)
+
+
+def _mut_variance_no_d(qbar, cov, variant):
+    return np.einsum("...id,...de,...ie->...i", qbar, cov, qbar) if variant == "exact" else \
+        np.einsum("...id,...d->...i", qbar * qbar, np.diagonal(cov, axis1=-2, axis2=-1))
+
+
+def _mut_variance_diag_everywhere(qbar, cov, variant):
+    return np.einsum("...id,...d->...i", qbar * qbar, np.diagonal(cov, axis1=-2, axis2=-1)) / qbar.shape[-1]
+
+
+def _mut_threshold_variance_not_std(qbar, kbar, beta, variant="exact"):
+    d = qbar.shape[-1]
+    m, cov = ref.key_moments(kbar)
+    return np.einsum("...id,...d->...i", qbar, m) / math.sqrt(d) + beta * ref.threshold_variance(qbar, cov, variant)
+
+
+def _mut_gaussian_keep_no_top(sbar, theta):
+    return sbar >= theta[..., None]
+
+
 MUTANTS = {
     "pool divides by block size": ("pool", _mut_pool_by_blk),
     "proxy without 1/sqrt(d)": ("proxy", _mut_proxy_unscaled),
@@ -323,6 +425,11 @@ MUTANTS = {
     "correction with summed value": ("correction_terms", _mut_corr_summed_value),
     "pseudo-keys missing from denominator": ("attend_block", _mut_attend_no_pseudo_den),
     "exact logits scaled by 1/d": ("attend_block", _mut_attend_scale_d),
+    "key covariance normalised by nKB - 1": ("key_moments", _mut_moments_sample),
+    "threshold variance without 1/d": ("threshold_variance", _mut_variance_no_d),
+    "exact threshold from the diagonal only": ("threshold_variance", _mut_variance_diag_everywhere),
+    "threshold uses the variance, not sigma": ("gaussian_threshold", _mut_threshold_variance_not_std),
+    "top block not forced": ("gaussian_keep", _mut_gaussian_keep_no_top),
 }
 
 
