@@ -75,6 +75,10 @@ struct FwdParams {
   const int *order;                   // fetch order of the work items, or null (item order)
   int *status;                        // device status word
   unsigned long long timeout_ns;      // limit of every device-side wait
+  // Query-dependent Gaussian threshold per (b, h, query block), or null: with it a block
+  // is kept iff its proxy is >= theta (and the row's top block always), in place of the
+  // running-max rule with tau.
+  const float *theta;
 };
 
 template <int D_, int BK_, int SUBQ_>
@@ -214,9 +218,13 @@ struct VecOf<2> {
 // time, and the 32 per-block dot products of a chunk are finished with one
 // transpose-sum. The attention kernel's router and the planning kernel both route
 // through this function, so they take identical decisions.
+// Routes query block qb: sets the keep bits in msk and, when `correct`, accumulates the
+// correction of the dropped blocks. Returns the number of kept blocks; top_j receives the
+// block with the largest proxy (lowest index on ties; Gaussian threshold only), and
+// force_j (>= 0) is kept whatever its proxy.
 template <int D, int BQ, int BK>
-__device__ __forceinline__ void route_scan(const FwdParams &p, int bh, int qb, int lane, bool correct, uint32_t *msk,
-                                           float (&cacc)[D / 32], float &lacc, float &M) {
+__device__ __forceinline__ int route_scan(const FwdParams &p, int bh, int qb, int lane, bool correct, uint32_t *msk,
+                                          float (&cacc)[D / 32], float &lacc, float &M, int force_j, int &top_j) {
   constexpr int VPL = D / 32;  // dimensions per lane
   using V = VecOf<VPL>;
   using VecT = typename V::T;
@@ -237,6 +245,11 @@ __device__ __forceinline__ void route_scan(const FwdParams &p, int bh, int qb, i
 #pragma unroll
   for (int e = 0; e < VPL; ++e) cacc[e] = 0.f;
   lacc = 0.f;
+  const bool gauss = p.theta != nullptr;
+  const float th = gauss ? __ldg(p.theta + static_cast<size_t>(bh) * p.nQB + qb) : 0.f;
+  int kept = 0;
+  float top_s = -CUDART_INF_F;
+  top_j = nKB;
 
   for (int t0 = 0; t0 < nKB; t0 += 32) {
     float part[32];
@@ -268,9 +281,27 @@ __device__ __forceinline__ void route_scan(const FwdParams &p, int bh, int qb, i
       if (lane >= off) m = fmaxf(m, y);
     }
     m = fmaxf(m, M);
-    const bool keep = valid && (s >= m - p.tau);
+    const bool keep = valid && (gauss ? (s >= th || j == force_j) : (s >= m - p.tau));
     const float Mn = __shfl_sync(0xffffffffu, m, 31);
     if (keep) atomicOr(&msk[j >> 5], 1u << (j & 31));
+    kept += __popc(__ballot_sync(0xffffffffu, keep));
+    if (gauss) {
+      float bs = valid ? s : -CUDART_INF_F;
+      int bj = valid ? j : nKB;
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        const float os = __shfl_xor_sync(0xffffffffu, bs, off);
+        const int oj = __shfl_xor_sync(0xffffffffu, bj, off);
+        if (os > bs || (os == bs && oj < bj)) {
+          bs = os;
+          bj = oj;
+        }
+      }
+      if (bs > top_s || (bs == top_s && bj < top_j)) {
+        top_s = bs;
+        top_j = bj;
+      }
+    }
     if (correct) {
       if (Mn > M) {
         const float f = expf(M - Mn);  // 0 on the first chunk (M = -inf)
@@ -309,6 +340,22 @@ __device__ __forceinline__ void route_scan(const FwdParams &p, int bh, int qb, i
   }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) lacc += __shfl_xor_sync(0xffffffffu, lacc, off);
+  return kept;
+}
+
+// route_scan under either rule. Under the Gaussian threshold a query block whose proxies
+// all fall below its threshold keeps its top block: the scan is repeated with that block
+// forced (the correction sums of the first scan included it as dropped).
+template <int D, int BQ, int BK>
+__device__ __forceinline__ int route_block(const FwdParams &p, int bh, int qb, int lane, bool correct, uint32_t *msk,
+                                           float (&cacc)[D / 32], float &lacc, float &M) {
+  int top_j = 0;
+  int kept = route_scan<D, BQ, BK>(p, bh, qb, lane, correct, msk, cacc, lacc, M, -1, top_j);
+  if (p.theta && kept == 0) {
+    int unused = 0;
+    kept = route_scan<D, BQ, BK>(p, bh, qb, lane, correct, msk, cacc, lacc, M, top_j, unused);
+  }
+  return kept;
 }
 
 template <class C>
@@ -318,7 +365,7 @@ __device__ __forceinline__ void route_query_block(SmemCtl<C> &sc, RouteSlot<C> &
   const bool correct = (p.mode == 2);
   float cacc[VPL];
   float lacc, M;
-  route_scan<C::D, C::BQ, C::BK>(p, bh, qb, lane, correct, sc.mask[sb], cacc, lacc, M);
+  route_block<C::D, C::BQ, C::BK>(p, bh, qb, lane, correct, sc.mask[sb], cacc, lacc, M);
 #pragma unroll
   for (int e = 0; e < VPL; ++e) rs.Cv[sb][lane * VPL + e] = correct ? cacc[e] : 0.f;
   if (lane == 0) {
@@ -954,6 +1001,122 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
   }
 }
 
+// ------------------------------------------------------------------ Gaussian threshold
+
+// Pooled-key moments of one (b, h) over its key blocks (equal weight, 1/nKB): the mean
+// m[D] and the covariance C[D][D] (diag = 0) or only its diagonal (diag = 1), written to
+// kmom[bh] = {m, C or diag(C)}. One CTA per (b, h), 256 threads; the covariance is
+// accumulated as 16 x 16 thread tiles of (D/16)^2 entries over 32-row chunks of the
+// centred pooled keys staged in shared memory.
+template <int D>
+__global__ void __launch_bounds__(256) gauss_moments_kernel(const float *kbar, float *kmom, int nKB, int diag) {
+  constexpr int T = D / 16;
+  __shared__ float mean[D];
+  __shared__ float rows[32][D];
+  const int bh = blockIdx.x;
+  const float *kb = kbar + static_cast<size_t>(bh) * nKB * D;
+  float *out = kmom + static_cast<size_t>(bh) * (D + D * D);
+  const float inv_n = 1.f / static_cast<float>(nKB);
+  for (int e = threadIdx.x; e < D; e += blockDim.x) {
+    float a = 0.f;
+    for (int j = 0; j < nKB; ++j) a += kb[static_cast<size_t>(j) * D + e];
+    mean[e] = a * inv_n;
+    out[e] = a * inv_n;
+  }
+  __syncthreads();
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  float acc[T][T];
+#pragma unroll
+  for (int a = 0; a < T; ++a)
+#pragma unroll
+    for (int b = 0; b < T; ++b) acc[a][b] = 0.f;
+  for (int j0 = 0; j0 < nKB; j0 += 32) {
+    for (int x = threadIdx.x; x < 32 * D; x += blockDim.x) {
+      const int r = x / D, e = x - r * D;
+      rows[r][e] = (j0 + r < nKB) ? kb[static_cast<size_t>(j0 + r) * D + e] - mean[e] : 0.f;
+    }
+    __syncthreads();
+    for (int r = 0; r < 32; ++r) {
+      float ra[T], rb[T];
+#pragma unroll
+      for (int a = 0; a < T; ++a) ra[a] = rows[r][ty * T + a];
+#pragma unroll
+      for (int b = 0; b < T; ++b) rb[b] = rows[r][tx * T + b];
+      if (diag) {
+        if (tx == ty) {
+#pragma unroll
+          for (int a = 0; a < T; ++a) acc[a][a] = fmaf(ra[a], ra[a], acc[a][a]);
+        }
+      } else {
+#pragma unroll
+        for (int a = 0; a < T; ++a)
+#pragma unroll
+          for (int b = 0; b < T; ++b) acc[a][b] = fmaf(ra[a], rb[b], acc[a][b]);
+      }
+    }
+    __syncthreads();
+  }
+  float *c = out + D;
+  if (diag) {
+    if (tx == ty) {
+#pragma unroll
+      for (int a = 0; a < T; ++a) c[ty * T + a] = acc[a][a] * inv_n;
+    }
+  } else {
+#pragma unroll
+    for (int a = 0; a < T; ++a)
+#pragma unroll
+      for (int b = 0; b < T; ++b) c[(ty * T + a) * D + tx * T + b] = acc[a][b] * inv_n;
+  }
+}
+
+// theta_i = mu_i + beta * sigma_i per query block: mu_i = q_i . m / sqrt(D) and
+// sigma_i^2 = q_i^T C q_i / D (or sum_e q_ie^2 C_ee / D). Grid (ceil(nQB / 8), B*H), one
+// warp per query block; C is staged in shared memory with a padded row stride.
+template <int D>
+__global__ void __launch_bounds__(256) gauss_theta_kernel(const float *qbar, const float *kmom, float *theta,
+                                                          int nQB, float beta, int diag) {
+  extern __shared__ float cs[];  // [D][D + 1] (exact) or [D] (diag), then q rows [8][D]
+  const int bh = blockIdx.y;
+  const float *mom = kmom + static_cast<size_t>(bh) * (D + D * D);
+  const int ncov = diag ? D : D * D;
+  float *cov = cs;
+  float *qs = cs + (diag ? D : D * (D + 1));
+  for (int x = threadIdx.x; x < ncov; x += blockDim.x) cov[diag ? x : (x / D) * (D + 1) + (x % D)] = mom[D + x];
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int i = blockIdx.x * 8 + warp;
+  if (i >= nQB) return;
+  const float *qr = qbar + (static_cast<size_t>(bh) * nQB + i) * D;
+  float *q = qs + warp * D;
+  for (int e = lane; e < D; e += 32) q[e] = qr[e];
+  __syncwarp();
+  float mu = 0.f, var = 0.f;
+  for (int e = lane; e < D; e += 32) {
+    mu = fmaf(q[e], mom[e], mu);
+    if (diag) {
+      var = fmaf(q[e] * q[e], cov[e], var);
+    } else {
+      float y = 0.f;
+      const float *row = cov + e * (D + 1);
+      for (int b = 0; b < D; ++b) y = fmaf(row[b], q[b], y);
+      var = fmaf(q[e], y, var);
+    }
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    mu += __shfl_xor_sync(0xffffffffu, mu, off);
+    var += __shfl_xor_sync(0xffffffffu, var, off);
+  }
+  if (lane == 0) {
+    float t;
+    if (beta == -CUDART_INF_F) t = -CUDART_INF_F;
+    else if (beta == CUDART_INF_F) t = CUDART_INF_F;
+    else t = mu * rsqrtf(static_cast<float>(D)) + beta * sqrtf(fmaxf(var / static_cast<float>(D), 0.f));
+    theta[static_cast<size_t>(bh) * nQB + i] = t;
+  }
+}
+
 // ------------------------------------------------------------------ planning pass
 
 // Work-item schedule for the attention kernel. Each warp routes one item (query tile)
@@ -983,7 +1146,7 @@ __global__ void __launch_bounds__(256) plan_kernel(const FwdParams p, int *cost,
     float lacc, M;
     for (int sb = 0; sb < SUBQ; ++sb) {
       const int qb = tile * SUBQ + sb;
-      if (qb < p.nQB) route_scan<D, BQ, BK>(p, bh, qb, lane, false, mask[warp][sb], cacc, lacc, M);
+      if (qb < p.nQB) route_block<D, BQ, BK>(p, bh, qb, lane, false, mask[warp][sb], cacc, lacc, M);
     }
     __syncwarp();
     int cnt = 0;

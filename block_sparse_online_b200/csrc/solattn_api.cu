@@ -27,7 +27,7 @@ int nblocks(int N, int blk) { return (N + blk - 1) / blk; }
 bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 struct WsLayout {
-  size_t qbar, kbar, vbar, v16, cost, order, total;
+  size_t qbar, kbar, vbar, v16, cost, order, kmom, theta, total;
 };
 
 int check_shape(int B, int H, int N, int d, int Bq, int Bk) {
@@ -49,7 +49,9 @@ WsLayout ws_layout(int B, int H, int N, int d, int Bq, int Bk) {
   const size_t items = bh * static_cast<size_t>(nblocks(N, 128));  // one work item per 128-row tile
   w.cost = w.v16 + align_up(bh * N * d * 2, kAlign);
   w.order = w.cost + align_up(items * sizeof(int), kAlign);
-  w.total = w.order + align_up(items * sizeof(int), kAlign);
+  w.kmom = w.order + align_up(items * sizeof(int), kAlign);  // pooled-key moments (Gaussian threshold)
+  w.theta = w.kmom + align_up(bh * (d + static_cast<size_t>(d) * d) * sizeof(float), kAlign);
+  w.total = w.theta + align_up(bh * nblocks(N, Bq) * sizeof(float), kAlign);
   return w;
 }
 
@@ -208,19 +210,47 @@ int noalloc_scratch(void **out) {
   return SOLATTN_OK;
 }
 
+// Pooled-key moments per (b, h), then the threshold of every query block.
+template <int D>
+int launch_threshold_d(const float *qbar, const float *kbar, float *kmom, float *theta, int BH, int nQB, int nKB,
+                       float beta, bool diag, cudaStream_t st) {
+  gauss_moments_kernel<D><<<BH, 256, 0, st>>>(kbar, kmom, nKB, diag ? 1 : 0);
+  if (cudaGetLastError() != cudaSuccess) return SOLATTN_ECUDA;
+  const size_t smem = sizeof(float) * ((diag ? D : D * (D + 1)) + 8 * D);
+  if (cudaFuncSetAttribute(gauss_theta_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess)
+    return SOLATTN_ECUDA;
+  gauss_theta_kernel<D><<<dim3((nQB + 7) / 8, BH), 256, smem, st>>>(qbar, kmom, theta, nQB, beta, diag ? 1 : 0);
+  if (cudaGetLastError() != cudaSuccess) return SOLATTN_ECUDA;
+  return SOLATTN_OK;
+}
+int launch_threshold(int d, const float *qbar, const float *kbar, float *kmom, float *theta, int BH, int nQB, int nKB,
+                     float beta, bool diag, cudaStream_t st) {
+  return d == 64 ? launch_threshold_d<64>(qbar, kbar, kmom, theta, BH, nQB, nKB, beta, diag, st)
+                 : launch_threshold_d<128>(qbar, kbar, kmom, theta, BH, nQB, nKB, beta, diag, st);
+}
+
 int items_total(int B, int H, int N) {
   // One work item per 128-row query tile.
   return B * H * ((N + 127) / 128);
 }
 
+// Routing rule of a forward call: the running maximum with tau, or the query-dependent
+// Gaussian threshold with beta (exact covariance or its diagonal).
+enum Rule { kRunningMax = 0, kGaussExact = 1, kGaussDiag = 2 };
+
 int forward_impl(const void *q, const void *k, const void *v, void *out, int B, int H, int N, int d, int Bq, int Bk,
                  float tau, int mode, const solattn_stats *stats, void *workspace, size_t ws_bytes, void *stream,
-                 void *ev_attn_begin, void *ev_attn_end) {
+                 void *ev_attn_begin, void *ev_attn_end, int rule = kRunningMax, float beta = 0.f) {
   if (!q || !k || !v || !out || !stats || !stats->kept_per_head) return SOLATTN_EINVAL;
   const int rc = check_shape(B, H, N, d, Bq, Bk);
   if (rc != SOLATTN_OK) return rc;
   if (mode < SOLATTN_DENSE || mode > SOLATTN_KEEP_CORRECT) return SOLATTN_EINVAL;
-  if (!(tau >= 0.f)) return SOLATTN_EINVAL;  // negative or NaN
+  if (rule == kRunningMax) {
+    if (!(tau >= 0.f)) return SOLATTN_EINVAL;  // negative or NaN
+  } else if (beta != beta) {
+    return SOLATTN_EINVAL;  // NaN
+  }
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16)) return SOLATTN_EINVAL;
   if (!aligned(stats->kept_per_head, 8) || (stats->keep_mask && !aligned(stats->keep_mask, 4)))
     return SOLATTN_EINVAL;
@@ -284,6 +314,14 @@ int forward_impl(const void *q, const void *k, const void *v, void *out, int B, 
   p.timeout_ns = kDefaultTimeoutNs;
   p.items_per_head = nblocks(N, 128);
   p.order = nullptr;
+  p.theta = nullptr;
+  if (mode != SOLATTN_DENSE && rule != kRunningMax) {
+    float *kmom = reinterpret_cast<float *>(ws + wl.kmom);
+    float *theta = reinterpret_cast<float *>(ws + wl.theta);
+    const int rt = launch_threshold(d, qbar, kbar, kmom, theta, BH, nQB, nKB, beta, rule == kGaussDiag, st);
+    if (rt != SOLATTN_OK) return rt;
+    p.theta = theta;
+  }
   if (mode != SOLATTN_DENSE) {
     // Schedule: heads in groups whose K and V16 fit in ~64 MB of L2 together, costliest
     // tiles first within a group.
@@ -356,6 +394,14 @@ int solattn_forward_noalloc(const void *q, const void *k, const void *v, void *o
   // stream before its kernels run, and overwrites every pooled block it reads.
   return forward_impl(q, k, v, out, B, H, N, d, Bq, Bk, tau, mode, stats, scratch, kNoAllocScratchBytes, stream,
                       nullptr, nullptr);
+}
+
+int solattn_forward_gaussian(const void *q, const void *k, const void *v, void *out, int B, int H, int N, int d,
+                             int Bq, int Bk, float beta, int variant, int mode, const solattn_stats *stats,
+                             void *workspace, size_t ws_bytes, void *stream) {
+  if (variant != SOLATTN_GAUSS_EXACT && variant != SOLATTN_GAUSS_DIAG) return SOLATTN_EINVAL;
+  return forward_impl(q, k, v, out, B, H, N, d, Bq, Bk, 0.f, mode, stats, workspace, ws_bytes, stream, nullptr,
+                      nullptr, variant == SOLATTN_GAUSS_EXACT ? kGaussExact : kGaussDiag, beta);
 }
 
 int solattn_get_status(const void *workspace, void *stream) {

@@ -29,7 +29,8 @@ MAX_KEY_BLOCKS = 1024
 EXPORTS = ("solattn_workspace_size", "solattn_pool", "solattn_forward", "solattn_forward_events",
            "solattn_get_status",
            "solattn_host_workspace_size", "solattn_forward_host", "solattn_watchdog_selftest",
-           "solattn_selftest_exp2", "solattn_forward_noalloc", "solattn_strerror")
+           "solattn_selftest_exp2", "solattn_forward_noalloc", "solattn_forward_gaussian", "solattn_strerror")
+GAUSS_VARIANTS = {"exact": 0, "diag": 1}  # solattn_gauss_variant
 
 
 class SolAttnError(RuntimeError):
@@ -57,6 +58,9 @@ def _load():
     lib.solattn_forward.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, f, i, ctypes.POINTER(_Stats), vp, sz, vp]
     lib.solattn_forward.restype = i
     lib.solattn_forward_events.argtypes = lib.solattn_forward.argtypes + [vp, vp]
+    lib.solattn_forward_gaussian.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, ctypes.POINTER(_Stats),
+                                             vp, sz, vp]
+    lib.solattn_forward_gaussian.restype = i
     lib.solattn_forward_events.restype = i
     lib.solattn_forward_host.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp, vp, sz, vp]
     lib.solattn_forward_host.restype = i
@@ -132,19 +136,8 @@ def solattn_pool(x: torch.Tensor, blk: int, out: torch.Tensor | None = None, str
     return out
 
 
-def solattn_forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, Bq: int, Bk: int, tau: float,
-                    mode="keep_correct", out: torch.Tensor | None = None,
-                    kept_per_head: torch.Tensor | None = None, keep_mask: bool | torch.Tensor = False,
-                    workspace: torch.Tensor | None = None, stream=None, events=None):
-    """Run the Sol-Attn forward operator on bf16 [B, H, N, d] CUDA tensors.
-
-    ``events``: optional pair of ``torch.cuda.Event(enable_timing=True)`` recorded
-    around the attention kernel (solattn_forward_events).
-
-    Returns (out bf16 [B, H, N, d], kept_per_head int64 [B, H], keep_mask uint32
-    [B, H, nQB, ceil(nKB/32)] or None). Asynchronous on ``stream``; device-side
-    errors are reported by :func:`solattn_get_status` on the workspace.
-    """
+def _prepare(q, k, v, Bq, Bk, out, kept_per_head, keep_mask, workspace):
+    """Checks the inputs and allocates what the caller did not pass."""
     B, H, N, d = _bhnd(q)
     for t in (q, k, v):
         if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous() or tuple(t.shape) != (B, H, N, d):
@@ -163,6 +156,24 @@ def solattn_forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, Bq: int, 
     if workspace is None:
         workspace = alloc_workspace(B, H, N, d, Bq, Bk, dev)
     stats = _Stats(kept_per_head.data_ptr(), mask.data_ptr() if mask is not None else None)
+    return B, H, N, d, out, kept_per_head, mask, workspace, stats
+
+
+def solattn_forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, Bq: int, Bk: int, tau: float,
+                    mode="keep_correct", out: torch.Tensor | None = None,
+                    kept_per_head: torch.Tensor | None = None, keep_mask: bool | torch.Tensor = False,
+                    workspace: torch.Tensor | None = None, stream=None, events=None):
+    """Run the Sol-Attn forward operator on bf16 [B, H, N, d] CUDA tensors.
+
+    ``events``: optional pair of ``torch.cuda.Event(enable_timing=True)`` recorded
+    around the attention kernel (solattn_forward_events).
+
+    Returns (out bf16 [B, H, N, d], kept_per_head int64 [B, H], keep_mask uint32
+    [B, H, nQB, ceil(nKB/32)] or None). Asynchronous on ``stream``; device-side
+    errors are reported by :func:`solattn_get_status` on the workspace.
+    """
+    B, H, N, d, out, kept_per_head, mask, workspace, stats = _prepare(q, k, v, Bq, Bk, out, kept_per_head,
+                                                                      keep_mask, workspace)
     args = (q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, H, N, d, Bq, Bk,
             ctypes.c_float(float(tau)), _mode(mode), ctypes.byref(stats), workspace.data_ptr(),
             workspace.numel(), _stream(stream))
@@ -176,6 +187,25 @@ def solattn_forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, Bq: int, 
         rc = _lib.solattn_forward_events(*args, ctypes.c_void_p(events[0].cuda_event),
                                          ctypes.c_void_p(events[1].cuda_event))
     _check(rc, "solattn_forward")
+    return out, kept_per_head, mask
+
+
+def solattn_forward_gaussian(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, Bq: int, Bk: int, beta: float,
+                             variant="exact", mode="keep_correct", out: torch.Tensor | None = None,
+                             kept_per_head: torch.Tensor | None = None, keep_mask: bool | torch.Tensor = False,
+                             workspace: torch.Tensor | None = None, stream=None):
+    """The forward operator under the query-dependent Gaussian threshold
+    (theta_i = mu_i + beta * sigma_i; ``variant`` "exact" or "diag"). Returns what
+    :func:`solattn_forward` returns."""
+    if variant not in GAUSS_VARIANTS:
+        raise ValueError(f"unknown variant {variant!r}")
+    B, H, N, d, out, kept_per_head, mask, workspace, stats = _prepare(q, k, v, Bq, Bk, out, kept_per_head,
+                                                                      keep_mask, workspace)
+    rc = _lib.solattn_forward_gaussian(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, H, N, d, Bq,
+                                       Bk, ctypes.c_float(float(beta)), GAUSS_VARIANTS[variant], _mode(mode),
+                                       ctypes.byref(stats), workspace.data_ptr(), workspace.numel(),
+                                       _stream(stream))
+    _check(rc, "solattn_forward_gaussian")
     return out, kept_per_head, mask
 
 

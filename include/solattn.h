@@ -172,6 +172,35 @@ int solattn_forward_noalloc(const void *q, const void *k, const void *v, void *o
                             int B, int H, int N, int d, int Bq, int Bk, float tau, int mode,
                             const solattn_stats *stats, void *stream);
 
+/* Variant of the Gaussian threshold's variance estimate. */
+typedef enum {
+  SOLATTN_GAUSS_EXACT = 0,  /* full pooled-key covariance: sigma_i^2 = q_i^T Cov[K] q_i / d      */
+  SOLATTN_GAUSS_DIAG = 1    /* its diagonal only: sigma_i^2 = sum_e q_ie^2 Cov[K]_ee / d          */
+} solattn_gauss_variant;
+
+/*
+ * solattn_forward with the pages' query-dependent Gaussian threshold in place of the
+ * running-maximum rule ("Sol-Attn: Accelerating Video Generation Inference via
+ * On-the-Fly Attention Sparsification", paperlayer summary §2, Figure 2: a threshold from
+ * the proxy-logit mean, standard deviation and a standardized offset beta; §3
+ * "Dynamic threshold routing": mean and variance from the pooled keys' first and second
+ * moments, one shared cutoff; appendix "Diagonal threshold estimator").
+ *
+ *   theta_i  = q_i . E[K] / sqrt(d) + beta * sigma_i, with E and Cov taken over the key
+ *              blocks' pooled rows k_j (equal weight, 1/nKB), sigma_i as in `variant`
+ *   keep     iff s_ij >= theta_i; the block with query block i's largest proxy (lowest
+ *              index on ties) is always kept, so no exact set is empty
+ *   output   as solattn_forward for `mode` (dense ignores beta)
+ *
+ * beta may be +-infinity (-inf keeps every block, +inf only each row's top block).
+ * Errors: beta NaN or an unknown variant -> SOLATTN_EINVAL; otherwise as
+ * solattn_forward. The workspace is the same (solattn_workspace_size).
+ */
+int solattn_forward_gaussian(const void *q, const void *k, const void *v, void *out,
+                             int B, int H, int N, int d, int Bq, int Bk, float beta, int variant,
+                             int mode, const solattn_stats *stats, void *workspace, size_t ws_bytes,
+                             void *stream);
+
 /*
  * Synchronise `stream` and read the device status word of `workspace`
  * (SOLATTN_OK, or SOLATTN_ETIMEOUT if a bounded device-side wait gave up).

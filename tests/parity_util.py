@@ -31,26 +31,35 @@ def unpack_mask(mask: torch.Tensor, nKB: int) -> np.ndarray:
     return bits[..., :nKB].astype(bool)
 
 
-def run_gpu(q, k, v, Bq, Bk, tau, mode):
+def run_gpu(q, k, v, Bq, Bk, tau, mode, gauss=None):
+    """gauss: None (running-max rule with tau) or (beta, variant) for the Gaussian threshold."""
     from block_sparse_online_b200 import solattn
     dev = torch.device("cuda:0")
     qd, kd, vd = (t.to(dev).contiguous() for t in (q, k, v))
     ws = solattn.alloc_workspace(*qd.shape, Bq, Bk, dev)
-    out, kept, mask = solattn.solattn_forward(qd, kd, vd, Bq, Bk, tau, mode, keep_mask=True, workspace=ws)
+    if gauss is None:
+        out, kept, mask = solattn.solattn_forward(qd, kd, vd, Bq, Bk, tau, mode, keep_mask=True, workspace=ws)
+    else:
+        out, kept, mask = solattn.solattn_forward_gaussian(qd, kd, vd, Bq, Bk, gauss[0], gauss[1], mode,
+                                                           keep_mask=True, workspace=ws)
     st = solattn.solattn_get_status(ws)
     assert st == 0, f"device status {st}"
     torch.cuda.synchronize()
     return out.cpu(), kept.cpu(), mask
 
 
-def check_case(q, k, v, Bq, Bk, tau, mode, qblocks=None, label=""):
+def check_case(q, k, v, Bq, Bk, tau, mode, qblocks=None, label="", gauss=None):
     """Run one case on the GPU and compare keep sets, counts and outputs with the oracle.
-    Returns a dict of the measured errors."""
+    gauss: None (running-max rule with tau) or (beta, variant). Returns a dict of the
+    measured errors."""
     B, H, N, d = q.shape
     nQB, nKB = -(-N // Bq), -(-N // Bk)
-    out, kept, mask = run_gpu(q, k, v, Bq, Bk, tau, mode)
+    out, kept, mask = run_gpu(q, k, v, Bq, Bk, tau, mode, gauss)
     gpu_keep = unpack_mask(mask, nKB)
-    ref_keep, margin, _ = ref.keep_sets(q, k, Bq, Bk, tau, mode)
+    if gauss is None:
+        ref_keep, margin, _ = ref.keep_sets(q, k, Bq, Bk, tau, mode)
+    else:
+        ref_keep, margin, _ = ref.keep_sets_gaussian(q, k, Bq, Bk, gauss[0], gauss[1], mode)
     diff = gpu_keep != ref_keep
     flips = int(diff.sum())
     if flips:

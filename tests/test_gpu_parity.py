@@ -175,3 +175,51 @@ def test_software_exp2_within_bound():
     # far below the clamp the result is a tiny positive number (zero once packed to fp16)
     tiny = solattn.solattn_selftest_exp2(torch.tensor([-200.0, -1e30], device="cuda")).cpu()
     assert (tiny >= 0).all() and (tiny < 1e-37).all()
+
+
+# ------------------------------------------------------------ query-dependent Gaussian threshold
+
+GAUSS_SHAPES = [
+    (1, 2, 1000, 64, 64, 64),
+    (1, 2, 777, 128, 128, 64),
+    (2, 1, 1300, 128, 64, 128),
+    (1, 3, 640, 128, 128, 128),
+]
+
+
+@pytest.mark.parametrize("variant", ("exact", "diag"))
+@pytest.mark.parametrize("mode", MODES)
+def test_gaussian_tiny(variant, mode):
+    q, k, v = synth.make_inputs("tiny")
+    for beta in (-INF, 0.0, 0.8, 1.5):
+        check_case(q, k, v, 64, 64, 0.0, mode, gauss=(beta, variant), label=f"tiny gauss {variant} {mode} {beta}")
+
+
+@pytest.mark.parametrize("shape", GAUSS_SHAPES, ids=[str(s) for s in GAUSS_SHAPES])
+@pytest.mark.parametrize("variant", ("exact", "diag"))
+def test_gaussian_shapes(shape, variant):
+    B, H, N, d, Bq, Bk = shape
+    cfg = synth.Config("adhoc", B=B, H=H, d=d, grid=(1, 1, N), Bq=Bq, Bk=Bk, taus=(), seed=31 + N)
+    q, k, v = synth.make_inputs(cfg)
+    for mode in ("keep_drop", "keep_correct"):
+        for beta in (0.5, 1.0, 2.5):
+            check_case(q, k, v, Bq, Bk, 0.0, mode, gauss=(beta, variant), label=f"{shape} gauss {variant} {mode} {beta}")
+
+
+def test_gaussian_top_block_only():
+    # beta = +inf: every query block keeps exactly its top block.
+    q, k, v = synth.make_inputs("tiny")
+    stats = check_case(q, k, v, 64, 64, 0.0, "keep_correct", gauss=(INF, "exact"), label="gauss +inf")
+    assert stats["flips"] == 0
+    out, kept, mask = run_gpu(q, k, v, 64, 64, 0.0, "keep_drop", gauss=(INF, "diag"))
+    assert (unpack_mask(mask, 16).sum(axis=-1) == 1).all()
+
+
+def test_gaussian_video480_config():
+    cfg = synth.CONFIGS["video480"]
+    q, k, v = synth.make_inputs(cfg)
+    blocks = sampled_blocks(cfg.B, cfg.H, cfg.N, cfg.Bq, cfg.Bk, 4, seed=cfg.seed)
+    for variant in ("exact", "diag"):
+        for mode, beta in (("keep_correct", 1.0), ("keep_drop", 1.5)):
+            check_case(q, k, v, cfg.Bq, cfg.Bk, 0.0, mode, qblocks=blocks, gauss=(beta, variant),
+                       label=f"video480 gauss {variant} {mode} {beta}")

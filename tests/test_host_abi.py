@@ -95,6 +95,38 @@ def test_forward_without_device_reports_cuda_error():
     assert _call() in (solattn.SOLATTN_ECUDA, solattn.SOLATTN_EUNSUPPORTED)
 
 
+def _call_gauss(beta=1.0, variant=0, mode=2, **kw):
+    """solattn_forward_gaussian with placeholder pointers (invalid cases only, as _call)."""
+    a = dict(q=4096, k=4096, v=4096, out=4096, B=1, H=1, N=256, d=128, Bq=128, Bk=128, kept=4096, mask=None,
+             ws=4096, ws_bytes=1 << 30)
+    a.update(kw)
+    st = solattn._Stats(a["kept"], a["mask"])
+    return solattn._lib.solattn_forward_gaussian(a["q"], a["k"], a["v"], a["out"], a["B"], a["H"], a["N"], a["d"],
+                                                 a["Bq"], a["Bk"], ctypes.c_float(beta), variant, mode,
+                                                 ctypes.byref(st), a["ws"], a["ws_bytes"], None)
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="placeholder pointers are used only without a GPU")
+@pytest.mark.parametrize("kw,want", [
+    (dict(beta=float("nan")), solattn.SOLATTN_EINVAL),
+    (dict(variant=2), solattn.SOLATTN_EINVAL),
+    (dict(variant=-1), solattn.SOLATTN_EINVAL),
+    (dict(mode=5), solattn.SOLATTN_EINVAL),
+    (dict(q=None), solattn.SOLATTN_EINVAL),
+    (dict(d=96), solattn.SOLATTN_EUNSUPPORTED),
+    (dict(ws_bytes=100), solattn.SOLATTN_EWORKSPACE),
+])
+def test_forward_gaussian_rejects_bad_arguments(kw, want):
+    assert _call_gauss(**kw) == want
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="placeholder pointers are used only without a GPU")
+def test_forward_gaussian_accepts_infinite_beta_and_negative_beta():
+    # +-inf and negative beta are valid; without a GPU the call fails only at the device query.
+    for beta in (float("inf"), float("-inf"), -1.5):
+        assert _call_gauss(beta=beta) in (solattn.SOLATTN_ECUDA, solattn.SOLATTN_EUNSUPPORTED)
+
+
 @pytest.mark.skipif(torch.cuda.is_available(), reason="placeholder pointers are used only without a GPU")
 def test_pool_rejects_bad_arguments():
     f = solattn._lib.solattn_pool
