@@ -54,8 +54,9 @@ constexpr float kLog2e = 1.4426950408889634f;
 // more than this many log2 units, so P stays <= 2^8 and O is rarely rescaled.
 constexpr float kRescaleSlack = 8.0f;
 // One pair of exponentials in this many is computed on the FMA pipe (polynomial)
-// instead of the MUFU unit, which the softmax otherwise saturates.
-constexpr int kPolyEvery = 4;
+// instead of the MUFU unit. Measured against 3, 4, 6 and none in the same run: 8 is the
+// fastest (the polynomial's extra instructions cost issue slots the softmax also needs).
+constexpr int kPolyEvery = 8;
 
 struct FwdParams {
   int N;
