@@ -35,6 +35,8 @@ n_i = |R_i|; key blocks j with columns C_j, n_j = |C_j|; d = head dim):
    "Approximation error"); keep_drop drops the dropped-block terms (abstract,
    "keep-or-drop sparsification"); dense keeps every block.
 6. Stats: kept blocks per (b, h) = sum over query blocks of |K_i|.
+7. Sinks (optional): the key blocks holding the first n_sink key tokens are kept by
+   every query block (text tokens retained as sinks in the exact branch).
 
 All arithmetic is float64 on the exact bf16 input values.
 """
@@ -141,12 +143,29 @@ def route_row(s_row: np.ndarray, visit: np.ndarray, tau: float):
     return keep, margin
 
 
-def keep_sets(q, k, Bq: int, Bk: int, tau: float, mode="keep_correct", order: str = "rotated"):
+def sink_blocks(n_sink: int, Bk: int) -> int:
+    """Key blocks that hold any of the first n_sink key tokens (text tokens kept as sinks in
+    the exact branch: paperlayer summary, App. A Additional Experimental Details). Reading:
+    the sinks are a prefix of the key sequence and the blocks overlapping it are kept whole."""
+    return -(-int(n_sink) // Bk)
+
+
+def apply_sinks(keep: np.ndarray, margin: np.ndarray, n_sink: int, Bk: int):
+    """Every query block keeps the sink blocks (margin +inf: no threshold decides them)."""
+    ns = sink_blocks(n_sink, Bk)
+    if ns:
+        keep[..., :ns] = True
+        margin[..., :ns] = np.inf
+    return keep, margin
+
+
+def keep_sets(q, k, Bq: int, Bk: int, tau: float, mode="keep_correct", order: str = "rotated", n_sink: int = 0):
     """Keep sets of every query block.
 
     Returns (keep [B, H, nQB, nKB] bool, margin [B, H, nQB, nKB] float64,
     sbar [B, H, nQB, nKB] float64). In dense mode every block is kept and the
-    margin is +inf.
+    margin is +inf. The sink blocks of ``n_sink`` leading key tokens are kept too; their
+    proxies still enter the running maximum, so the other decisions do not change.
     """
     mode = _mode_name(mode)
     q = as_f64(q)
@@ -163,6 +182,7 @@ def keep_sets(q, k, Bq: int, Bk: int, tau: float, mode="keep_correct", order: st
         for b in range(B):
             for h in range(H):
                 keep[b, h, i], margin[b, h, i] = route_row(sbar[b, h, i], visit, tau)
+    keep, margin = apply_sinks(keep, margin, n_sink, Bk)
     return keep, margin, sbar
 
 
@@ -208,7 +228,7 @@ def attend_block(q_rows, k, v, kept_cols, pseudo):
 
 
 def forward(q, k, v, Bq: int, Bk: int, tau: float, mode="keep_correct", order: str = "rotated",
-            keep: np.ndarray | None = None, qblocks=None):
+            keep: np.ndarray | None = None, qblocks=None, n_sink: int = 0):
     """Sol-Attn output in float64.
 
     q, k, v: [B, H, N, d] (bf16 torch tensors or arrays; converted exactly).
@@ -223,7 +243,7 @@ def forward(q, k, v, Bq: int, Bk: int, tau: float, mode="keep_correct", order: s
     B, H, N, d = q.shape
     nQB, nKB = n_blocks(N, Bq), n_blocks(N, Bk)
     if keep is None:
-        keep, _, sbar = keep_sets(q, k, Bq, Bk, tau, mode, order)
+        keep, _, sbar = keep_sets(q, k, Bq, Bk, tau, mode, order, n_sink)
     else:
         keep = np.asarray(keep, dtype=bool)
         sbar = proxy(pool(q, Bq), pool(k, Bk))
@@ -288,15 +308,20 @@ def gaussian_threshold(qbar: np.ndarray, kbar: np.ndarray, beta: float, variant:
     return mu + beta * sigma
 
 
-def gaussian_keep(sbar: np.ndarray, theta: np.ndarray) -> np.ndarray:
-    """Keep iff s_ij >= theta_i, plus the row's top block: [..., nQB, nKB] bool."""
+def gaussian_keep(sbar: np.ndarray, theta: np.ndarray, n_sink_blocks: int = 0) -> np.ndarray:
+    """Keep iff s_ij >= theta_i, plus the sink blocks; a row left empty keeps its top
+    block: [..., nQB, nKB] bool."""
     keep = sbar >= theta[..., None]
+    keep[..., :n_sink_blocks] = True
     top = np.argmax(sbar, axis=-1)
-    np.put_along_axis(keep, top[..., None], True, axis=-1)
-    return keep
+    empty = ~keep.any(axis=-1)
+    top_keep = np.zeros_like(keep)
+    np.put_along_axis(top_keep, top[..., None], True, axis=-1)
+    return keep | (top_keep & empty[..., None])
 
 
-def keep_sets_gaussian(q, k, Bq: int, Bk: int, beta: float, variant: str = "exact", mode="keep_correct"):
+def keep_sets_gaussian(q, k, Bq: int, Bk: int, beta: float, variant: str = "exact", mode="keep_correct",
+                       n_sink: int = 0):
     """Keep sets under the Gaussian threshold.
 
     Returns (keep, margin = s - theta (+inf for a top block kept only because it is
@@ -311,17 +336,18 @@ def keep_sets_gaussian(q, k, Bq: int, Bk: int, beta: float, variant: str = "exac
     if mode == "dense" or beta == -math.inf:
         return np.ones(sbar.shape, dtype=bool), np.full(sbar.shape, np.inf), sbar
     theta = gaussian_threshold(qbar, kbar, beta, variant)
-    keep = gaussian_keep(sbar, theta)
+    keep = gaussian_keep(sbar, theta, sink_blocks(n_sink, Bk))
     margin = sbar - theta[..., None]
     margin = np.where(keep & (margin < 0), np.inf, margin)
+    keep, margin = apply_sinks(keep, margin, n_sink, Bk)
     return keep, margin, sbar
 
 
 def forward_gaussian(q, k, v, Bq: int, Bk: int, beta: float, variant: str = "exact", mode="keep_correct",
-                     keep: np.ndarray | None = None, qblocks=None):
+                     keep: np.ndarray | None = None, qblocks=None, n_sink: int = 0):
     """Output under the Gaussian threshold (steps 1, 2 and 5 as in ``forward``)."""
     if keep is None:
-        keep, _, _ = keep_sets_gaussian(q, k, Bq, Bk, beta, variant, mode)
+        keep, _, _ = keep_sets_gaussian(q, k, Bq, Bk, beta, variant, mode, n_sink)
     return forward(q, k, v, Bq, Bk, 0.0, mode, keep=keep, qblocks=qblocks)
 
 

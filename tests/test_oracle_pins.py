@@ -326,8 +326,27 @@ def pin_gaussian_limits_and_monotone():
     assert np.abs(t_ex - t_dg).max() > 1e-3
 
 
+def pin_sinks():
+    # Sinks add exactly the leading ceil(n_sink / Bk) key blocks to every keep set and
+    # change nothing else (their proxies already entered the running max).
+    q, k, v = _rand(1, 2, 777, 16, seed=12)
+    base, _, sbar = ref.keep_sets(q, k, 64, 64, 1.0, "keep_drop")
+    for n_sink, nb in ((1, 1), (64, 1), (65, 2), (200, 4)):
+        got, margin, _ = ref.keep_sets(q, k, 64, 64, 1.0, "keep_drop", n_sink=n_sink)
+        assert got[..., :nb].all() and np.isinf(margin[..., :nb]).all()
+        np.testing.assert_array_equal(got[..., nb:], base[..., nb:])
+        g2, _, _ = ref.keep_sets_gaussian(q, k, 64, 64, 3.0, "exact", n_sink=n_sink)
+        assert g2[..., :nb].all()
+    # every key token a sink: keep_drop is dense attention, by SDPA
+    out, _ = ref.forward(q, k, v, 64, 64, 1.0, "keep_drop", n_sink=777)
+    np.testing.assert_allclose(out, _sdpa(q, k, v), rtol=1e-9, atol=1e-9)
+    # a Gaussian row with sinks but nothing over its threshold keeps only the sinks
+    g3, _, _ = ref.keep_sets_gaussian(q, k, 64, 64, 1e9, "diag", n_sink=10)
+    assert (g3.sum(axis=-1) == 1).all() and g3[..., 0].all()
+
+
 PINS += [pin_gaussian_matches_row_statistics, pin_gaussian_diagonal_design, pin_gaussian_keep_fraction,
-         pin_gaussian_limits_and_monotone]
+         pin_gaussian_limits_and_monotone, pin_sinks]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
@@ -411,8 +430,14 @@ def _mut_threshold_variance_not_std(qbar, kbar, beta, variant="exact"):
     return np.einsum("...id,...d->...i", qbar, m) / math.sqrt(d) + beta * ref.threshold_variance(qbar, cov, variant)
 
 
-def _mut_gaussian_keep_no_top(sbar, theta):
-    return sbar >= theta[..., None]
+def _mut_gaussian_keep_no_top(sbar, theta, n_sink_blocks=0):
+    keep = sbar >= theta[..., None]
+    keep[..., :n_sink_blocks] = True
+    return keep
+
+
+def _mut_sink_blocks_floor(n_sink, Bk):
+    return int(n_sink) // Bk
 
 
 MUTANTS = {
@@ -430,6 +455,7 @@ MUTANTS = {
     "exact threshold from the diagonal only": ("threshold_variance", _mut_variance_diag_everywhere),
     "threshold uses the variance, not sigma": ("gaussian_threshold", _mut_threshold_variance_not_std),
     "top block not forced": ("gaussian_keep", _mut_gaussian_keep_no_top),
+    "sink blocks rounded down": ("sink_blocks", _mut_sink_blocks_floor),
 }
 
 
