@@ -80,6 +80,8 @@ struct FwdParams {
   // is kept iff its proxy is >= theta (and the row's top block always), in place of the
   // running-max rule with tau.
   const float *theta;
+  // Key blocks 0 .. n_sink_blocks - 1 hold sink tokens: kept by every query block.
+  int n_sink_blocks;
 };
 
 template <int D_, int BK_, int SUBQ_>
@@ -248,6 +250,7 @@ __device__ __forceinline__ int route_scan(const FwdParams &p, int bh, int qb, in
   lacc = 0.f;
   const bool gauss = p.theta != nullptr;
   const float th = gauss ? __ldg(p.theta + static_cast<size_t>(bh) * p.nQB + qb) : 0.f;
+  const int nsb = p.n_sink_blocks;  // sink blocks are kept outright
   int kept = 0;
   float top_s = -CUDART_INF_F;
   top_j = nKB;
@@ -282,7 +285,8 @@ __device__ __forceinline__ int route_scan(const FwdParams &p, int bh, int qb, in
       if (lane >= off) m = fmaxf(m, y);
     }
     m = fmaxf(m, M);
-    const bool keep = valid && (gauss ? (s >= th || j == force_j) : (s >= m - p.tau));
+    const float thr = gauss ? th : m - p.tau;
+    const bool keep = valid && (s >= thr || j == force_j || j < nsb);
     const float Mn = __shfl_sync(0xffffffffu, m, 31);
     if (keep) atomicOr(&msk[j >> 5], 1u << (j & 31));
     kept += __popc(__ballot_sync(0xffffffffu, keep));

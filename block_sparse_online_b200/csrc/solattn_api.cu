@@ -241,7 +241,8 @@ enum Rule { kRunningMax = 0, kGaussExact = 1, kGaussDiag = 2 };
 
 int forward_impl(const void *q, const void *k, const void *v, void *out, int B, int H, int N, int d, int Bq, int Bk,
                  float tau, int mode, const solattn_stats *stats, void *workspace, size_t ws_bytes, void *stream,
-                 void *ev_attn_begin, void *ev_attn_end, int rule = kRunningMax, float beta = 0.f) {
+                 void *ev_attn_begin, void *ev_attn_end, int rule = kRunningMax, float beta = 0.f,
+                 int n_sink = 0) {
   if (!q || !k || !v || !out || !stats || !stats->kept_per_head) return SOLATTN_EINVAL;
   const int rc = check_shape(B, H, N, d, Bq, Bk);
   if (rc != SOLATTN_OK) return rc;
@@ -251,6 +252,7 @@ int forward_impl(const void *q, const void *k, const void *v, void *out, int B, 
   } else if (beta != beta) {
     return SOLATTN_EINVAL;  // NaN
   }
+  if (n_sink < 0 || n_sink > N) return SOLATTN_EINVAL;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16)) return SOLATTN_EINVAL;
   if (!aligned(stats->kept_per_head, 8) || (stats->keep_mask && !aligned(stats->keep_mask, 4)))
     return SOLATTN_EINVAL;
@@ -315,6 +317,7 @@ int forward_impl(const void *q, const void *k, const void *v, void *out, int B, 
   p.items_per_head = nblocks(N, 128);
   p.order = nullptr;
   p.theta = nullptr;
+  p.n_sink_blocks = nblocks(n_sink, Bk);
   if (mode != SOLATTN_DENSE && rule != kRunningMax) {
     float *kmom = reinterpret_cast<float *>(ws + wl.kmom);
     float *theta = reinterpret_cast<float *>(ws + wl.theta);
@@ -402,6 +405,21 @@ int solattn_forward_gaussian(const void *q, const void *k, const void *v, void *
   if (variant != SOLATTN_GAUSS_EXACT && variant != SOLATTN_GAUSS_DIAG) return SOLATTN_EINVAL;
   return forward_impl(q, k, v, out, B, H, N, d, Bq, Bk, 0.f, mode, stats, workspace, ws_bytes, stream, nullptr,
                       nullptr, variant == SOLATTN_GAUSS_EXACT ? kGaussExact : kGaussDiag, beta);
+}
+
+int solattn_forward_ex(const void *q, const void *k, const void *v, void *out, int B, int H, int N, int d, int Bq,
+                       int Bk, const solattn_route *route, int mode, const solattn_stats *stats, void *workspace,
+                       size_t ws_bytes, void *stream) {
+  if (!route) return SOLATTN_EINVAL;
+  int rule;
+  switch (route->rule) {
+    case SOLATTN_RULE_RUNNING_MAX: rule = kRunningMax; break;
+    case SOLATTN_RULE_GAUSS_EXACT: rule = kGaussExact; break;
+    case SOLATTN_RULE_GAUSS_DIAG: rule = kGaussDiag; break;
+    default: return SOLATTN_EINVAL;
+  }
+  return forward_impl(q, k, v, out, B, H, N, d, Bq, Bk, route->tau, mode, stats, workspace, ws_bytes, stream, nullptr,
+                      nullptr, rule, route->beta, route->n_sink);
 }
 
 int solattn_get_status(const void *workspace, void *stream) {

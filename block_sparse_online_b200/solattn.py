@@ -29,8 +29,10 @@ MAX_KEY_BLOCKS = 1024
 EXPORTS = ("solattn_workspace_size", "solattn_pool", "solattn_forward", "solattn_forward_events",
            "solattn_get_status",
            "solattn_host_workspace_size", "solattn_forward_host", "solattn_watchdog_selftest",
-           "solattn_selftest_exp2", "solattn_forward_noalloc", "solattn_forward_gaussian", "solattn_strerror")
+           "solattn_selftest_exp2", "solattn_forward_noalloc", "solattn_forward_gaussian", "solattn_forward_ex",
+           "solattn_strerror")
 GAUSS_VARIANTS = {"exact": 0, "diag": 1}  # solattn_gauss_variant
+RULES = {"running_max": 0, "gauss_exact": 1, "gauss_diag": 2}  # solattn_rule
 
 
 class SolAttnError(RuntimeError):
@@ -41,6 +43,10 @@ class SolAttnError(RuntimeError):
 
 class _Stats(ctypes.Structure):
     _fields_ = [("kept_per_head", ctypes.c_void_p), ("keep_mask", ctypes.c_void_p)]
+
+
+class _Route(ctypes.Structure):  # solattn_route
+    _fields_ = [("rule", ctypes.c_int), ("tau", ctypes.c_float), ("beta", ctypes.c_float), ("n_sink", ctypes.c_int)]
 
 
 def _load():
@@ -61,6 +67,9 @@ def _load():
     lib.solattn_forward_gaussian.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, ctypes.POINTER(_Stats),
                                              vp, sz, vp]
     lib.solattn_forward_gaussian.restype = i
+    lib.solattn_forward_ex.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, ctypes.POINTER(_Route), i,
+                                       ctypes.POINTER(_Stats), vp, sz, vp]
+    lib.solattn_forward_ex.restype = i
     lib.solattn_forward_events.restype = i
     lib.solattn_forward_host.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp, vp, sz, vp]
     lib.solattn_forward_host.restype = i
@@ -206,6 +215,25 @@ def solattn_forward_gaussian(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, 
                                        ctypes.byref(stats), workspace.data_ptr(), workspace.numel(),
                                        _stream(stream))
     _check(rc, "solattn_forward_gaussian")
+    return out, kept_per_head, mask
+
+
+def solattn_forward_ex(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, Bq: int, Bk: int, mode="keep_correct",
+                       rule="running_max", tau: float = 0.0, beta: float = 0.0, n_sink: int = 0,
+                       out: torch.Tensor | None = None, kept_per_head: torch.Tensor | None = None,
+                       keep_mask: bool | torch.Tensor = False, workspace: torch.Tensor | None = None, stream=None):
+    """The forward operator with every routing option: ``rule`` "running_max" (tau),
+    "gauss_exact" or "gauss_diag" (beta), and ``n_sink`` leading key tokens kept as sinks.
+    Returns what :func:`solattn_forward` returns."""
+    if rule not in RULES:
+        raise ValueError(f"unknown rule {rule!r}")
+    B, H, N, d, out, kept_per_head, mask, workspace, stats = _prepare(q, k, v, Bq, Bk, out, kept_per_head,
+                                                                      keep_mask, workspace)
+    route = _Route(RULES[rule], float(tau), float(beta), int(n_sink))
+    rc = _lib.solattn_forward_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, H, N, d, Bq, Bk,
+                                 ctypes.byref(route), _mode(mode), ctypes.byref(stats), workspace.data_ptr(),
+                                 workspace.numel(), _stream(stream))
+    _check(rc, "solattn_forward_ex")
     return out, kept_per_head, mask
 
 

@@ -201,6 +201,41 @@ int solattn_forward_gaussian(const void *q, const void *k, const void *v, void *
                              int mode, const solattn_stats *stats, void *workspace, size_t ws_bytes,
                              void *stream);
 
+/* Routing rule of solattn_forward_ex. */
+typedef enum {
+  SOLATTN_RULE_RUNNING_MAX = 0,  /* keep iff s_ij >= M - tau (solattn_forward)                 */
+  SOLATTN_RULE_GAUSS_EXACT = 1,  /* keep iff s_ij >= theta_i, exact covariance (solattn_forward_gaussian) */
+  SOLATTN_RULE_GAUSS_DIAG = 2    /* the same with the diagonal covariance                       */
+} solattn_rule;
+
+/* Routing options of solattn_forward_ex. */
+typedef struct {
+  int rule;    /* solattn_rule                                                          */
+  float tau;   /* running-max rule: tau >= 0 (+infinity keeps every block)              */
+  float beta;  /* Gaussian rules: standardized offset (not NaN; +-infinity allowed)     */
+  int n_sink;  /* leading key tokens kept as sinks: 0 <= n_sink <= N                    */
+} solattn_route;
+
+/*
+ * The forward operator with every routing option. Sinks: the text key-value tokens that
+ * the pages keep in the exact branch for every query ("Sol-Attn: Accelerating Video
+ * Generation Inference via On-the-Fly Attention Sparsification", paperlayer summary,
+ * App. A Additional Experimental Details). This library takes them to be the first
+ * n_sink key tokens (a prefix of the [B][H][N][d] layout): every key block that holds
+ * one of them, ceil(n_sink / Bk) blocks, is kept by every query block under either rule
+ * and is never folded into the correction. The proxies of sink blocks still enter the
+ * running maximum, so the other keep decisions do not change; under a Gaussian rule the
+ * top-block guard applies only to a query block that would otherwise keep nothing.
+ * With n_sink = 0, rule RUNNING_MAX equals solattn_forward and the Gaussian rules equal
+ * solattn_forward_gaussian.
+ * Errors: route NULL, an unknown rule, tau < 0 or NaN (running max), beta NaN (Gaussian)
+ * or n_sink outside [0, N] -> SOLATTN_EINVAL; otherwise as solattn_forward.
+ */
+int solattn_forward_ex(const void *q, const void *k, const void *v, void *out,
+                       int B, int H, int N, int d, int Bq, int Bk, const solattn_route *route,
+                       int mode, const solattn_stats *stats, void *workspace, size_t ws_bytes,
+                       void *stream);
+
 /*
  * Synchronise `stream` and read the device status word of `workspace`
  * (SOLATTN_OK, or SOLATTN_ETIMEOUT if a bounded device-side wait gave up).

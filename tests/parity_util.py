@@ -31,13 +31,19 @@ def unpack_mask(mask: torch.Tensor, nKB: int) -> np.ndarray:
     return bits[..., :nKB].astype(bool)
 
 
-def run_gpu(q, k, v, Bq, Bk, tau, mode, gauss=None):
-    """gauss: None (running-max rule with tau) or (beta, variant) for the Gaussian threshold."""
+def run_gpu(q, k, v, Bq, Bk, tau, mode, gauss=None, n_sink=0):
+    """gauss: None (running-max rule with tau) or (beta, variant) for the Gaussian threshold;
+    n_sink > 0 goes through solattn_forward_ex."""
     from block_sparse_online_b200 import solattn
     dev = torch.device("cuda:0")
     qd, kd, vd = (t.to(dev).contiguous() for t in (q, k, v))
     ws = solattn.alloc_workspace(*qd.shape, Bq, Bk, dev)
-    if gauss is None:
+    if n_sink:
+        rule = "running_max" if gauss is None else f"gauss_{gauss[1]}"
+        out, kept, mask = solattn.solattn_forward_ex(qd, kd, vd, Bq, Bk, mode, rule, tau=tau,
+                                                     beta=0.0 if gauss is None else gauss[0], n_sink=n_sink,
+                                                     keep_mask=True, workspace=ws)
+    elif gauss is None:
         out, kept, mask = solattn.solattn_forward(qd, kd, vd, Bq, Bk, tau, mode, keep_mask=True, workspace=ws)
     else:
         out, kept, mask = solattn.solattn_forward_gaussian(qd, kd, vd, Bq, Bk, gauss[0], gauss[1], mode,
@@ -48,18 +54,18 @@ def run_gpu(q, k, v, Bq, Bk, tau, mode, gauss=None):
     return out.cpu(), kept.cpu(), mask
 
 
-def check_case(q, k, v, Bq, Bk, tau, mode, qblocks=None, label="", gauss=None):
+def check_case(q, k, v, Bq, Bk, tau, mode, qblocks=None, label="", gauss=None, n_sink=0):
     """Run one case on the GPU and compare keep sets, counts and outputs with the oracle.
-    gauss: None (running-max rule with tau) or (beta, variant). Returns a dict of the
-    measured errors."""
+    gauss: None (running-max rule with tau) or (beta, variant); n_sink: sink tokens.
+    Returns a dict of the measured errors."""
     B, H, N, d = q.shape
     nQB, nKB = -(-N // Bq), -(-N // Bk)
-    out, kept, mask = run_gpu(q, k, v, Bq, Bk, tau, mode, gauss)
+    out, kept, mask = run_gpu(q, k, v, Bq, Bk, tau, mode, gauss, n_sink)
     gpu_keep = unpack_mask(mask, nKB)
     if gauss is None:
-        ref_keep, margin, _ = ref.keep_sets(q, k, Bq, Bk, tau, mode)
+        ref_keep, margin, _ = ref.keep_sets(q, k, Bq, Bk, tau, mode, n_sink=n_sink)
     else:
-        ref_keep, margin, _ = ref.keep_sets_gaussian(q, k, Bq, Bk, gauss[0], gauss[1], mode)
+        ref_keep, margin, _ = ref.keep_sets_gaussian(q, k, Bq, Bk, gauss[0], gauss[1], mode, n_sink=n_sink)
     diff = gpu_keep != ref_keep
     flips = int(diff.sum())
     if flips:

@@ -223,3 +223,32 @@ def test_gaussian_video480_config():
         for mode, beta in (("keep_correct", 1.0), ("keep_drop", 1.5)):
             check_case(q, k, v, cfg.Bq, cfg.Bk, 0.0, mode, qblocks=blocks, gauss=(beta, variant),
                        label=f"video480 gauss {variant} {mode} {beta}")
+
+
+# ------------------------------------------------------------ sink tokens (solattn_forward_ex)
+
+@pytest.mark.parametrize("rule", ("running_max", "gauss_exact", "gauss_diag"))
+def test_sinks(rule):
+    gauss = None if rule == "running_max" else (1.5, rule.split("_")[1])
+    for shape in ((1, 2, 1000, 64, 64, 64), (1, 2, 777, 128, 128, 64)):
+        B, H, N, d, Bq, Bk = shape
+        cfg = synth.Config("adhoc", B=B, H=H, d=d, grid=(1, 1, N), Bq=Bq, Bk=Bk, taus=(), seed=41 + N)
+        q, k, v = synth.make_inputs(cfg)
+        for n_sink in (1, 64, 100, N):
+            for mode in ("keep_drop", "keep_correct"):
+                stats = check_case(q, k, v, Bq, Bk, 1.0, mode, gauss=gauss, n_sink=n_sink,
+                                   label=f"{shape} sinks {rule} {n_sink} {mode}")
+                if n_sink == N:
+                    assert stats["keep_ratio"] == 1.0
+
+
+def test_forward_ex_without_sinks_matches_the_other_entry_points():
+    from block_sparse_online_b200 import solattn
+    q, k, v = (t.cuda() for t in synth.make_inputs("tiny"))
+    a = solattn.solattn_forward(q, k, v, 64, 64, 2.0, "keep_correct")
+    b = solattn.solattn_forward_ex(q, k, v, 64, 64, "keep_correct", "running_max", tau=2.0)
+    c = solattn.solattn_forward_gaussian(q, k, v, 64, 64, 1.0, "diag", "keep_drop")
+    e = solattn.solattn_forward_ex(q, k, v, 64, 64, "keep_drop", "gauss_diag", beta=1.0)
+    torch.cuda.synchronize()
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+    assert torch.equal(c[0], e[0]) and torch.equal(c[1], e[1])
