@@ -37,6 +37,8 @@ n_i = |R_i|; key blocks j with columns C_j, n_j = |C_j|; d = head dim):
 6. Stats: kept blocks per (b, h) = sum over query blocks of |K_i|.
 7. Sinks (optional): the key blocks holding the first n_sink key tokens are kept by
    every query block (text tokens retained as sinks in the exact branch).
+8. Token-to-block correction (optional): the dropped block's pseudo-key logit is
+   q_r . k_j / sqrt(d) for each row r instead of the block proxy s_ij.
 
 All arithmetic is float64 on the exact bf16 input values.
 """
@@ -205,39 +207,57 @@ def correction_terms(sbar_row: np.ndarray, dropped: np.ndarray, counts: np.ndarr
     return sbar_row[idx], counts[idx].astype(np.float64), vbar[idx]
 
 
+def correction_terms_token(q_rows: np.ndarray, kbar: np.ndarray, dropped: np.ndarray, counts: np.ndarray,
+                           vbar: np.ndarray):
+    """Token-to-block pseudo-keys of the dropped blocks of one query block: the logit of
+    row r is q_r . k_j / sqrt(d) with the pooled key k_j (paperlayer summary §3
+    Methodology, "Unified execution": a token-to-block score tile determines the approximate
+    correction). Returns (logits [n_i, m], multiplicities [m], values [m, d])."""
+    idx = np.nonzero(dropped)[0]
+    d = q_rows.shape[-1]
+    return (q_rows @ kbar[idx].T) / math.sqrt(d), counts[idx].astype(np.float64), vbar[idx]
+
+
 def attend_block(q_rows, k, v, kept_cols, pseudo):
     """Closed-form weighted softmax of one query block.
 
     q_rows [n_i, d]; k, v [N, d]; kept_cols: bool [N]; pseudo = (logits,
-    multiplicities, values) of the pseudo-keys or None.
+    multiplicities, values) of the pseudo-keys or None; the logits are one per pseudo-key
+    ([m], the same for every row) or one per row and pseudo-key ([n_i, m]).
     """
     d = q_rows.shape[-1]
     s = (q_rows @ k[kept_cols].T) / math.sqrt(d)          # [n_i, n_kept]
     m = s.max(axis=1) if s.shape[1] else np.full(q_rows.shape[0], -np.inf)
-    if pseudo is not None and pseudo[0].size:
-        m = np.maximum(m, pseudo[0].max())
+    has_pseudo = pseudo is not None and pseudo[0].size
+    if has_pseudo:
+        logits = np.broadcast_to(pseudo[0], (q_rows.shape[0], pseudo[1].shape[0]))
+        m = np.maximum(m, logits.max(axis=1))
     e = np.exp(s - m[:, None])
     num = e @ v[kept_cols]
     den = e.sum(axis=1)
-    if pseudo is not None and pseudo[0].size:
-        logits, mult, vals = pseudo
-        w = mult[None, :] * np.exp(logits[None, :] - m[:, None])   # [n_i, m]
+    if has_pseudo:
+        _, mult, vals = pseudo
+        w = mult[None, :] * np.exp(logits - m[:, None])   # [n_i, m]
         num = num + w @ vals
         den = den + w.sum(axis=1)
     return num / den[:, None]
 
 
 def forward(q, k, v, Bq: int, Bk: int, tau: float, mode="keep_correct", order: str = "rotated",
-            keep: np.ndarray | None = None, qblocks=None, n_sink: int = 0):
+            keep: np.ndarray | None = None, qblocks=None, n_sink: int = 0, correction: str = "block"):
     """Sol-Attn output in float64.
 
     q, k, v: [B, H, N, d] (bf16 torch tensors or arrays; converted exactly).
     keep: optional [B, H, nQB, nKB] override of the keep sets (used to compare
     outputs on the GPU's own keep set where a near-threshold proxy flipped).
     qblocks: None for every query block, or an iterable of (b, h, i) triples.
+    correction: "block" (pseudo-key logit s_ij, the same for every row of query block i)
+    or "token" (logit q_r . k_j / sqrt(d) per row r).
     Returns (out [B, H, N, d] float64 with NaN rows for query blocks that were
     not computed, keep [B, H, nQB, nKB]).
     """
+    if correction not in ("block", "token"):
+        raise ValueError(correction)
     mode = _mode_name(mode)
     q, k, v = as_f64(q), as_f64(k), as_f64(v)
     B, H, N, d = q.shape
@@ -251,6 +271,7 @@ def forward(q, k, v, Bq: int, Bk: int, tau: float, mode="keep_correct", order: s
         keep = np.ones_like(keep)
     counts = valid_counts(N, Bk)
     vbar = pool(v, Bk) if mode == "keep_correct" else None
+    kbar = pool(k, Bk) if (mode == "keep_correct" and correction == "token") else None
     col_block = np.arange(N) // Bk
     out = np.full(q.shape, np.nan)
     if qblocks is None:
@@ -259,7 +280,9 @@ def forward(q, k, v, Bq: int, Bk: int, tau: float, mode="keep_correct", order: s
         rows = block_rows(N, Bq, i)
         kept_cols = keep[b, h, i][col_block]
         pseudo = None
-        if mode == "keep_correct":
+        if mode == "keep_correct" and correction == "token":
+            pseudo = correction_terms_token(q[b, h, rows], kbar[b, h], ~keep[b, h, i], counts, vbar[b, h])
+        elif mode == "keep_correct":
             pseudo = correction_terms(sbar[b, h, i], ~keep[b, h, i], counts, vbar[b, h])
         out[b, h, rows] = attend_block(q[b, h, rows], k[b, h], v[b, h], kept_cols, pseudo)
     return out, keep
@@ -344,11 +367,11 @@ def keep_sets_gaussian(q, k, Bq: int, Bk: int, beta: float, variant: str = "exac
 
 
 def forward_gaussian(q, k, v, Bq: int, Bk: int, beta: float, variant: str = "exact", mode="keep_correct",
-                     keep: np.ndarray | None = None, qblocks=None, n_sink: int = 0):
+                     keep: np.ndarray | None = None, qblocks=None, n_sink: int = 0, correction: str = "block"):
     """Output under the Gaussian threshold (steps 1, 2 and 5 as in ``forward``)."""
     if keep is None:
         keep, _, _ = keep_sets_gaussian(q, k, Bq, Bk, beta, variant, mode, n_sink)
-    return forward(q, k, v, Bq, Bk, 0.0, mode, keep=keep, qblocks=qblocks)
+    return forward(q, k, v, Bq, Bk, 0.0, mode, keep=keep, qblocks=qblocks, correction=correction)
 
 
 def sample_qblocks(B, H, nQB, Bq, Bk, nKB, per_head=64, seed=0):

@@ -345,8 +345,46 @@ def pin_sinks():
     assert (g3.sum(axis=-1) == 1).all() and g3[..., 0].all()
 
 
+def pin_token_correction():
+    N, d, blk = 700, 16, 64
+    rng = np.random.default_rng(17)
+    nb = -(-N // blk)
+    # (1) K constant inside each key block: the token-to-block pseudo-key reproduces every
+    # dropped block exactly, so keep_correct equals dense attention for any tau.
+    kb = rng.standard_normal((1, 2, nb, d)) * 0.8
+    k = np.repeat(kb, blk, axis=2)[:, :, :N]
+    q = rng.standard_normal((1, 2, N, d))
+    v = rng.standard_normal((1, 2, N, d))
+    dense = _sdpa(q, k, v)
+    for tau in (0.0, 0.05, 0.15):  # the proxies here span about 0.4: these taus drop blocks
+        out, keep = ref.forward(q, k, v, blk, blk, tau, "keep_correct", correction="token")
+        assert (~keep).any()
+        np.testing.assert_allclose(out, dense, rtol=1e-9, atol=1e-10)
+    # (2) Q constant inside each query block: token and block corrections coincide.
+    qb = rng.standard_normal((1, 2, nb, d))
+    qc = np.repeat(qb, blk, axis=2)[:, :, :N]
+    kr = rng.standard_normal((1, 2, N, d))
+    a, _ = ref.forward(qc, kr, v, blk, blk, 1.0, "keep_correct", correction="token")
+    b, _ = ref.forward(qc, kr, v, blk, blk, 1.0, "keep_correct", correction="block")
+    np.testing.assert_allclose(a, b, rtol=1e-11, atol=1e-12)
+    # (3) SDPA over the kept keys plus the dropped blocks' pooled keys, biased by log n_j.
+    q, k, v = _rand(1, 1, 300, 8, seed=23)
+    out, keep = ref.forward(q, k, v, 64, 64, 1.0, "keep_correct", correction="token")
+    kbar, vbar = ref.pool(k, 64), ref.pool(v, 64)
+    counts = ref.valid_counts(300, 64)
+    for i in range(keep.shape[2]):
+        rows = slice(i * 64, min(300, i * 64 + 64))
+        cols = keep[0, 0, i][np.arange(300) // 64]
+        drop = np.nonzero(~keep[0, 0, i])[0]
+        kk = np.concatenate([k[0, 0, cols], kbar[0, 0, drop]])
+        vv = np.concatenate([v[0, 0, cols], vbar[0, 0, drop]])
+        bias = np.concatenate([np.zeros(cols.sum()), np.log(counts[drop])])
+        want = _sdpa(q[:, :, rows], kk[None, None], vv[None, None], np.broadcast_to(bias, (1, 1, rows.stop - rows.start, kk.shape[0])).copy())
+        np.testing.assert_allclose(out[:, :, rows], want, rtol=1e-9, atol=1e-10)
+
+
 PINS += [pin_gaussian_matches_row_statistics, pin_gaussian_diagonal_design, pin_gaussian_keep_fraction,
-         pin_gaussian_limits_and_monotone, pin_sinks]
+         pin_gaussian_limits_and_monotone, pin_sinks, pin_token_correction]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
@@ -440,6 +478,20 @@ def _mut_sink_blocks_floor(n_sink, Bk):
     return int(n_sink) // Bk
 
 
+def _mut_token_uses_block_logit(q_rows, kbar, dropped, counts, vbar):
+    idx = np.nonzero(dropped)[0]
+    d = q_rows.shape[-1]
+    qbar = q_rows.mean(axis=0)
+    return np.broadcast_to((kbar[idx] @ qbar) / math.sqrt(d), (q_rows.shape[0], idx.size)), \
+        counts[idx].astype(np.float64), vbar[idx]
+
+
+def _mut_token_no_multiplicity(q_rows, kbar, dropped, counts, vbar):
+    idx = np.nonzero(dropped)[0]
+    d = q_rows.shape[-1]
+    return (q_rows @ kbar[idx].T) / math.sqrt(d), np.ones(idx.size), vbar[idx]
+
+
 MUTANTS = {
     "pool divides by block size": ("pool", _mut_pool_by_blk),
     "proxy without 1/sqrt(d)": ("proxy", _mut_proxy_unscaled),
@@ -456,6 +508,8 @@ MUTANTS = {
     "threshold uses the variance, not sigma": ("gaussian_threshold", _mut_threshold_variance_not_std),
     "top block not forced": ("gaussian_keep", _mut_gaussian_keep_no_top),
     "sink blocks rounded down": ("sink_blocks", _mut_sink_blocks_floor),
+    "token correction with the block logit": ("correction_terms_token", _mut_token_uses_block_logit),
+    "token correction without n_j": ("correction_terms_token", _mut_token_no_multiplicity),
 }
 
 
