@@ -401,6 +401,27 @@ def main():
                               "keep_ratio": round(float(b.mean()), 5),
                               "exec_tflops": round(ef / (ms * 1e-3) / 1e12, 2),
                               "dense_equiv_tflops": round(dense_flops / (ms * 1e-3) / 1e12, 2)})
+        # keep_correct with the token-to-block correction (pooled-key tiles on the tensor cores).
+        for tau in (3.0, 6.0):
+            _, _, m = solattn.solattn_forward_ex(qd, kd, vd, cfg.Bq, cfg.Bk, "keep_correct", tau=tau,
+                                                 correction="token", keep_mask=True, workspace=ws)
+            b = unpack(m, cfg.nKB)
+            ef = executed_flops(b, N, cfg.Bq, cfg.Bk, d)
+            ts = []
+            for i in range(8):
+                a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a0.record(stream)
+                solattn.solattn_forward_ex(qd, kd, vd, cfg.Bq, cfg.Bk, "keep_correct", tau=tau, correction="token",
+                                           out=out, kept_per_head=kept, workspace=ws)
+                a1.record(stream)
+                torch.cuda.synchronize()
+                if i >= 3:
+                    ts.append(a0.elapsed_time(a1))
+            ms = statistics.median(ts)
+            sweep.append({"mode": "keep_correct", "correction": "token", "tau": tau, "ms": round(ms, 4),
+                          "keep_ratio": round(float(b.mean()), 5),
+                          "exec_tflops": round(ef / (ms * 1e-3) / 1e12, 2),
+                          "dense_equiv_tflops": round(dense_flops / (ms * 1e-3) / 1e12, 2)})
         # The pages' query-dependent Gaussian threshold (theta = mu + beta * sigma), keep_correct.
         for variant in ("exact", "diag"):
             for beta in (0.5, 1.0, 1.5):

@@ -48,6 +48,10 @@ namespace solattn {
 
 constexpr int kMaxKeyBlocks = 1024;
 constexpr int kMaskWords = kMaxKeyBlocks / 32;
+// Token-to-block correction: the item's key stream ends with ceil(nKB / BK) tiles of the
+// head's pooled keys ("pseudo tiles"), flagged in the kept list.
+constexpr int kPseudoFlag = 0x8000;
+constexpr int kMaxPseudo = kMaxKeyBlocks / 64;
 constexpr int kStatusTimeout = -4;
 constexpr float kLog2e = 1.4426950408889634f;
 // Lazy rescaling: a row's reference max moves only when the tile max exceeds it by
@@ -82,6 +86,11 @@ struct FwdParams {
   const float *theta;
   // Key blocks 0 .. n_sink_blocks - 1 hold sink tokens: kept by every query block.
   int n_sink_blocks;
+  // keep_correct with the token-to-block correction: each row meets every dropped block
+  // as one pseudo-key (pooled key, logit q_r . k_j / sqrt(d), weight n_j, value v_j), fed
+  // to the tensor cores as n_pseudo tiles of pooled keys at the end of every item.
+  int token_corr;
+  int n_pseudo;
 };
 
 template <int D_, int BK_, int SUBQ_>
@@ -129,8 +138,10 @@ struct RouteSlot {
   float M[C::NSB];        // running proxy max (natural log units), -inf if no correction
   float L[C::NSB];        // sum over dropped j of n_j e^{s_ij - M}
   float Cv[C::NSB][C::D]; // sum over dropped j of n_j e^{s_ij - M} mean(V_j)
-  uint16_t jlist[kMaxKeyBlocks];  // kept key blocks (union over the item), ascending
-  uint8_t member[kMaxKeyBlocks];  // bit sb: query block sb of the item keeps jlist[u]
+  uint32_t kmask[C::NSB][kMaskWords];  // keep bits per query block (token-to-block correction)
+  uint16_t jlist[kMaxKeyBlocks + kMaxPseudo];  // kept key blocks (union over the item), ascending,
+                                               // then the pseudo tiles (kPseudoFlag | t)
+  uint8_t member[kMaxKeyBlocks + kMaxPseudo];  // bit sb: query block sb of the item keeps jlist[u]
 };
 
 template <class C>
@@ -367,7 +378,7 @@ template <class C>
 __device__ __forceinline__ void route_query_block(SmemCtl<C> &sc, RouteSlot<C> &rs, const FwdParams &p,
                                                   int bh, int sb, int qb, int lane) {
   constexpr int VPL = C::D / 32;
-  const bool correct = (p.mode == 2);
+  const bool correct = (p.mode == 2) && !p.token_corr;  // block-level correction sums
   float cacc[VPL];
   float lacc, M;
   route_block<C::D, C::BQ, C::BK>(p, bh, qb, lane, correct, sc.mask[sb], cacc, lacc, M);
@@ -471,10 +482,22 @@ __device__ void run_router(SmemCtl<C> &sc, const FwdParams &p, int lane) {
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) kept += __shfl_xor_sync(0xffffffffu, kept, off);
     __syncwarp();
+    int n_list = base;
+    if (p.mode == 2 && p.token_corr) {
+      // The pseudo tiles of the head's pooled keys, and the keep bits that mask them.
+      for (int sb = 0; sb < C::NSB; ++sb)
+        for (int w = lane; w < nW; w += 32) rs.kmask[sb][w] = sc.mask[sb][w];
+      for (int t = lane; t < p.n_pseudo; t += 32) {
+        rs.jlist[base + t] = static_cast<uint16_t>(kPseudoFlag | t);
+        rs.member[base + t] = static_cast<uint8_t>((1u << C::NSB) - 1u);
+      }
+      n_list += p.n_pseudo;
+    }
+    __syncwarp();
     if (lane == 0) {
       atomicAdd(p.kept_per_head + bh, kept);
       rs.item = item;
-      rs.n_union = base;
+      rs.n_union = n_list;
       mbar_arrive(&sc.route_full[s]);
     }
     __syncwarp();
@@ -486,7 +509,8 @@ __device__ void run_router(SmemCtl<C> &sc, const FwdParams &p, int lane) {
 
 template <class C>
 __device__ void run_producer(SmemCtl<C> &sc, const FwdParams &p, uint8_t *q_smem, uint8_t *ring,
-                             const CUtensorMap *tm_q, const CUtensorMap *tm_k, const CUtensorMap *tm_v) {
+                             const CUtensorMap *tm_q, const CUtensorMap *tm_k, const CUtensorMap *tm_v,
+                             const CUtensorMap *tm_kp, const CUtensorMap *tm_vp) {
   const volatile int *ab = &sc.abort_flag;
   uint32_t kv_it = 0, q_it = 0;
   bool ok = true;
@@ -500,10 +524,13 @@ __device__ void run_producer(SmemCtl<C> &sc, const FwdParams &p, uint8_t *q_smem
     }
     mbar_arrive_expect_tx(&sc.full[slot], C::KV_BYTES);
     uint8_t *dst = ring + slot * C::KV_BYTES;
+    // a pseudo tile is BK rows of the head's pooled keys / values (zero past nKB)
+    const bool pseudo = (j & kPseudoFlag) != 0;
+    const CUtensorMap *map = pseudo ? (is_v ? tm_vp : tm_kp) : (is_v ? tm_v : tm_k);
+    const int row = (j & (kPseudoFlag - 1)) * C::BK;
 #pragma unroll
     for (int pn = 0; pn < C::PANELS; ++pn)
-      tma_load_3d(smem_u32(dst + pn * (C::BK * 128)), is_v ? tm_v : tm_k, smem_u32(&sc.full[slot]), pn * 64,
-                  j * C::BK, bh);
+      tma_load_3d(smem_u32(dst + pn * (C::BK * 128)), map, smem_u32(&sc.full[slot]), pn * 64, row, bh);
     ++kv_it;
   };
   for (uint32_t r_it = 0;; ++r_it) {
@@ -693,7 +720,66 @@ __device__ void run_mma(SmemCtl<C> &sc, const FwdParams &p, uint32_t tmem, uint8
 
 // ------------------------------------------------------------------ softmax / epilogue
 
-template <class C>
+// Softmax of one pseudo tile of the head's pooled keys (token-to-block correction):
+// column c is key block jb = t * BK + c. It enters this row as one pseudo-key (logit
+// q_r . k_jb / sqrt(d), weight n_jb, value mean(V_jb)) only if jb exists and this row's
+// query block dropped it (bit clear in km). Kept out of line: it runs for a few tiles per
+// item and would otherwise add to the register pressure of the exact-block path.
+template <int BK>
+__device__ __noinline__ void softmax_pseudo_tile(uint32_t s_addr, int t, const uint32_t *km, int N, int nKB,
+                                                 float sc_log2, float &m_ref, float &alpha, float &lsum) {
+  constexpr int NCH = BK / 32;
+  const float lb = log2f(static_cast<float>(BK));
+  const float lb_last = log2f(static_cast<float>(N - (nKB - 1) * BK));
+  float mxs = -CUDART_INF_F;
+#pragma unroll 1
+  for (int c = 0; c < NCH; ++c) {
+    uint32_t xs[32];
+    tmem_ld32(s_addr + c * 32, xs);
+    tmem_wait_ld();
+    reg_fence32(xs);
+    const int jb0 = t * BK + c * 32;
+    const uint32_t kw = (jb0 < nKB) ? km[jb0 >> 5] : 0xffffffffu;  // past nKB: masked
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+      const int jb = jb0 + e;
+      if (jb < nKB && !((kw >> e) & 1u)) mxs = fmaxf(mxs, fmaf(__uint_as_float(xs[e]), sc_log2, jb == nKB - 1 ? lb_last : lb));
+    }
+  }
+  if (mxs > m_ref + kRescaleSlack) {
+    if (m_ref != -CUDART_INF_F) alpha = ex2_approx(m_ref - mxs);
+    m_ref = mxs;
+  }
+  const float neg_m = (m_ref == -CUDART_INF_F) ? 0.f : -m_ref;
+#pragma unroll 1
+  for (int c = 0; c < NCH; ++c) {
+    uint32_t xs[32];
+    tmem_ld32(s_addr + c * 32, xs);
+    tmem_wait_ld();
+    reg_fence32(xs);
+    const int jb0 = t * BK + c * 32;
+    const uint32_t kw = (jb0 < nKB) ? km[jb0 >> 5] : 0xffffffffu;
+    uint32_t pk[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      float pp[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int jb = jb0 + 2 * e + h;
+        const bool ok_col = jb < nKB && !((kw >> (2 * e + h)) & 1u);
+        const float bias = (jb == nKB - 1 ? lb_last : lb) + neg_m;
+        pp[h] = ok_col ? ex2_approx(fmaf(__uint_as_float(xs[2 * e + h]), sc_log2, bias)) : 0.f;
+      }
+      lsum += pp[0] + pp[1];
+      pk[e] = pack_f16x2(pp[0], pp[1]);
+    }
+    tmem_st16(s_addr + c * 16, pk);
+  }
+}
+
+// TOKEN: this instantiation handles pseudo tiles (token-to-block correction); the other
+// one has no such branch in its loop.
+template <class C, bool TOKEN>
 __device__ void run_softmax(SmemCtl<C> &sc, const FwdParams &p, uint32_t tmem, int w, int warp, int lane) {
   constexpr int BK = C::BK;
   constexpr int D = C::D;
@@ -744,111 +830,115 @@ __device__ void run_softmax(SmemCtl<C> &sc, const FwdParams &p, uint32_t tmem, i
         if (u >= w + 2) release(ring_index_v(u - 2, n));
         if (u + 2 >= n) mbar_arrive(&sc.q_empty[r_it % C::NQBUF]);
       }
-      // Two passes over the row of S, 32 columns per TMEM load, each load issued one chunk
-      // ahead: the row maximum (a tree of three-input max instructions per chunk), then the
-      // exponentials, whose fp16 pairs go back to TMEM 16 columns at a time. The reference
-      // max only moves when the row maximum exceeds it by more than the slack (O and l are
-      // then rescaled once, below).
-      constexpr int NCH = BK / 32;
-      const bool rk = (mem & row_bit) != 0;  // warp-uniform (a warp's rows share a query block)
-      const int ncol = (j == p.nKB - 1) ? (p.N - j * BK) : BK;
-      const bool full = rk && ncol == BK;    // no column of this block masked
-      float mx = -CUDART_INF_F;
-      uint32_t x[32];
-      if (rk) {
-        tmem_ld32(s_addr, x);
-        tmem_wait_ld();
-        reg_fence32(x);
-#pragma unroll
-        for (int c = 0; c < NCH; ++c) {
-          uint32_t y[32];
-          // the next chunk, or (after the last) chunk 0 again for the exponential pass; the
-          // fence keeps the arithmetic on this chunk after the load is issued
-          tmem_ld32(s_addr + ((c + 1) % NCH) * 32, y);
-          reg_fence32(x);
-          float m;
-          if (full) {
-            m = max_tree_bits<32>(x);
-          } else {
-            m = -CUDART_INF_F;
-#pragma unroll
-            for (int e = 0; e < 32; ++e)
-              if (c * 32 + e < ncol) m = fmaxf(m, u2f(x[e]));
-          }
-          mx = fmaxf(mx, m);
-          asm volatile("" ::"f"(mx));  // the tree stays ahead of the wait
-          tmem_wait_ld();
-          reg_fence32(y);
-#pragma unroll
-          for (int e = 0; e < 32; ++e) x[e] = y[e];
-        }
-      }
-      const float mxs = mx * sc_log2;
       float alpha = 1.f;  // rescale of this row's O and l for this S tile
-      if (mxs > m_ref + kRescaleSlack) {
-        if (m_ref != -CUDART_INF_F) alpha = ex2_approx(m_ref - mxs);
-        m_ref = mxs;
-      }
-      const float neg_m = (m_ref == -CUDART_INF_F) ? 0.f : -m_ref;
       float lsum = 0.f;
-      if (full) {
-        // Packed fp32 pairs; one pair in kPolyEvery goes through the FMA-pipe exp2.
-        const uint64_t scp = f2(sc_log2, sc_log2);
-        const uint64_t nmp = f2(neg_m, neg_m);
-        uint64_t acc = f2(0.f, 0.f);
-#pragma unroll
-        for (int c = 0; c < NCH; ++c) {
-          uint32_t y[32];
-          if (c + 1 < NCH) tmem_ld32(s_addr + (c + 1) * 32, y);
+      if (!TOKEN || !(j & kPseudoFlag)) {
+        // Two passes over the row of S, 32 columns per TMEM load, each load issued one chunk
+        // ahead: the row maximum (a tree of three-input max instructions per chunk), then the
+        // exponentials, whose fp16 pairs go back to TMEM 16 columns at a time. The reference
+        // max only moves when the row maximum exceeds it by more than the slack (O and l are
+        // then rescaled once, below).
+        constexpr int NCH = BK / 32;
+        const bool rk = (mem & row_bit) != 0;  // warp-uniform (a warp's rows share a query block)
+        const int ncol = (j == p.nKB - 1) ? (p.N - j * BK) : BK;
+        const bool full = rk && ncol == BK;    // no column of this block masked
+        float mx = -CUDART_INF_F;
+        uint32_t x[32];
+        if (rk) {
+          tmem_ld32(s_addr, x);
+          tmem_wait_ld();
           reg_fence32(x);
-          uint32_t pk[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const uint64_t xx = fma2(f2(u2f(x[2 * e]), u2f(x[2 * e + 1])), scp, nmp);
-            float x0, x1, p0, p1;
-            f2_split(xx, x0, x1);
-            if ((e % kPolyEvery) == kPolyEvery - 1) {
-              exp2_poly_x2(x0, x1, p0, p1);
+  #pragma unroll
+          for (int c = 0; c < NCH; ++c) {
+            uint32_t y[32];
+            // the next chunk, or (after the last) chunk 0 again for the exponential pass; the
+            // fence keeps the arithmetic on this chunk after the load is issued
+            tmem_ld32(s_addr + ((c + 1) % NCH) * 32, y);
+            reg_fence32(x);
+            float m;
+            if (full) {
+              m = max_tree_bits<32>(x);
             } else {
-              p0 = ex2_approx(x0);
-              p1 = ex2_approx(x1);
+              m = -CUDART_INF_F;
+  #pragma unroll
+              for (int e = 0; e < 32; ++e)
+                if (c * 32 + e < ncol) m = fmaxf(m, u2f(x[e]));
             }
-            acc = add2(acc, f2(p0, p1));
-            pk[e] = pack_f16x2(p0, p1);
-          }
-          tmem_st16(s_addr + c * 16, pk);
-          if (c + 1 < NCH) {
+            mx = fmaxf(mx, m);
+            asm volatile("" ::"f"(mx));  // the tree stays ahead of the wait
             tmem_wait_ld();
             reg_fence32(y);
-#pragma unroll
+  #pragma unroll
             for (int e = 0; e < 32; ++e) x[e] = y[e];
           }
         }
-        float s0, s1;
-        f2_split(acc, s0, s1);
-        lsum = s0 + s1;
-      } else {
-#pragma unroll
-        for (int c = 0; c < NCH; ++c) {
-          uint32_t y[32];
-          if (rk && c + 1 < NCH) tmem_ld32(s_addr + (c + 1) * 32, y);
-          uint32_t pk[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int col = c * 32 + 2 * e;
-            const float p0 = (rk && col < ncol) ? ex2_approx(fmaf(u2f(x[2 * e]), sc_log2, neg_m)) : 0.f;
-            const float p1 = (rk && col + 1 < ncol) ? ex2_approx(fmaf(u2f(x[2 * e + 1]), sc_log2, neg_m)) : 0.f;
-            lsum += p0 + p1;
-            pk[e] = pack_f16x2(p0, p1);
+        const float mxs = mx * sc_log2;
+        if (mxs > m_ref + kRescaleSlack) {
+          if (m_ref != -CUDART_INF_F) alpha = ex2_approx(m_ref - mxs);
+          m_ref = mxs;
+        }
+        const float neg_m = (m_ref == -CUDART_INF_F) ? 0.f : -m_ref;
+        if (full) {
+          // Packed fp32 pairs; one pair in kPolyEvery goes through the FMA-pipe exp2.
+          const uint64_t scp = f2(sc_log2, sc_log2);
+          const uint64_t nmp = f2(neg_m, neg_m);
+          uint64_t acc = f2(0.f, 0.f);
+  #pragma unroll
+          for (int c = 0; c < NCH; ++c) {
+            uint32_t y[32];
+            if (c + 1 < NCH) tmem_ld32(s_addr + (c + 1) * 32, y);
+            reg_fence32(x);
+            uint32_t pk[16];
+  #pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const uint64_t xx = fma2(f2(u2f(x[2 * e]), u2f(x[2 * e + 1])), scp, nmp);
+              float x0, x1, p0, p1;
+              f2_split(xx, x0, x1);
+              if ((e % kPolyEvery) == kPolyEvery - 1) {
+                exp2_poly_x2(x0, x1, p0, p1);
+              } else {
+                p0 = ex2_approx(x0);
+                p1 = ex2_approx(x1);
+              }
+              acc = add2(acc, f2(p0, p1));
+              pk[e] = pack_f16x2(p0, p1);
+            }
+            tmem_st16(s_addr + c * 16, pk);
+            if (c + 1 < NCH) {
+              tmem_wait_ld();
+              reg_fence32(y);
+  #pragma unroll
+              for (int e = 0; e < 32; ++e) x[e] = y[e];
+            }
           }
-          tmem_st16(s_addr + c * 16, pk);
-          if (rk && c + 1 < NCH) {
-            tmem_wait_ld();
-            reg_fence32(y);
-#pragma unroll
-            for (int e = 0; e < 32; ++e) x[e] = y[e];
+          float s0, s1;
+          f2_split(acc, s0, s1);
+          lsum = s0 + s1;
+        } else {
+  #pragma unroll
+          for (int c = 0; c < NCH; ++c) {
+            uint32_t y[32];
+            if (rk && c + 1 < NCH) tmem_ld32(s_addr + (c + 1) * 32, y);
+            uint32_t pk[16];
+  #pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const int col = c * 32 + 2 * e;
+              const float p0 = (rk && col < ncol) ? ex2_approx(fmaf(u2f(x[2 * e]), sc_log2, neg_m)) : 0.f;
+              const float p1 = (rk && col + 1 < ncol) ? ex2_approx(fmaf(u2f(x[2 * e + 1]), sc_log2, neg_m)) : 0.f;
+              lsum += p0 + p1;
+              pk[e] = pack_f16x2(p0, p1);
+            }
+            tmem_st16(s_addr + c * 16, pk);
+            if (rk && c + 1 < NCH) {
+              tmem_wait_ld();
+              reg_fence32(y);
+  #pragma unroll
+              for (int e = 0; e < 32; ++e) x[e] = y[e];
+            }
           }
         }
+      } else if constexpr (TOKEN) {
+        softmax_pseudo_tile<BK>(s_addr, j & (kPseudoFlag - 1), rs.kmask[sb], p.N, p.nKB, sc_log2, m_ref, alpha, lsum);
       }
       l = l * alpha + lsum;
       if (__any_sync(0xffffffffu, alpha != 1.f)) {
@@ -932,10 +1022,11 @@ __device__ void run_softmax(SmemCtl<C> &sc, const FwdParams &p, uint32_t tmem, i
 
 // ------------------------------------------------------------------ kernel
 
-template <class C>
+template <class C, bool TOKEN>
 __global__ void __launch_bounds__(C::NUM_THREADS, 1)
     solattn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                       const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kp,
+                       const __grid_constant__ CUtensorMap tm_vp, const FwdParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *q_smem = base;
@@ -973,6 +1064,10 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
+    if (p.token_corr) {
+      tma_prefetch_desc(&tm_kp);
+      tma_prefetch_desc(&tm_vp);
+    }
   }
   if (warp == 1) {
     tmem_alloc(&sc.tmem_base, C::TMEM_COLS);
@@ -986,7 +1081,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
   if (warp < C::CTRL_WARPS) {
     regs_dec<C::CTRL_REGS>();
     if (warp == 0) {
-      if (lane == 0) run_producer<C>(sc, p, q_smem, ring, &tm_q, &tm_k, &tm_v);
+      if (lane == 0) run_producer<C>(sc, p, q_smem, ring, &tm_q, &tm_k, &tm_v, &tm_kp, &tm_vp);
     } else if (warp == 1 || warp == 3) {
       if (lane == 0) run_mma<C>(sc, p, tmem, q_smem, ring, warp == 1 ? 0 : 1);
     } else if (warp == 2) {
@@ -994,7 +1089,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
     }
   } else {
     regs_inc<C::SOFTMAX_REGS>();
-    run_softmax<C>(sc, p, tmem, (warp - C::CTRL_WARPS) >> 2, warp, lane);
+    run_softmax<C, TOKEN>(sc, p, tmem, (warp - C::CTRL_WARPS) >> 2, warp, lane);
   }
 
   tc_fence_before_sync();

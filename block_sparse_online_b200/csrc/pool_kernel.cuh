@@ -83,4 +83,15 @@ __global__ void __launch_bounds__(128) pool_kernel(const PoolArgs args) {
   }
 }
 
+// bf16 copy of the pooled keys and fp16 copy of the pooled values ([B*H][nKB][d], same
+// layout as the fp32 arrays), the operands of the token-to-block correction tiles.
+__global__ void __launch_bounds__(256) pooled_copy_kernel(const float *kbar, const float *vbar, __nv_bfloat16 *k16,
+                                                          __half *v16, size_t n) {
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    k16[i] = __float2bfloat16_rn(kbar[i]);
+    v16[i] = __float2half_rn(vbar[i]);
+  }
+}
+
 }  // namespace solattn

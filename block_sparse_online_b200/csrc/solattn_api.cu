@@ -27,7 +27,7 @@ int nblocks(int N, int blk) { return (N + blk - 1) / blk; }
 bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 struct WsLayout {
-  size_t qbar, kbar, vbar, v16, cost, order, kmom, theta, total;
+  size_t qbar, kbar, vbar, v16, cost, order, kmom, theta, kbar16, vbar16, total;
 };
 
 int check_shape(int B, int H, int N, int d, int Bq, int Bk) {
@@ -51,7 +51,9 @@ WsLayout ws_layout(int B, int H, int N, int d, int Bq, int Bk) {
   w.order = w.cost + align_up(items * sizeof(int), kAlign);
   w.kmom = w.order + align_up(items * sizeof(int), kAlign);  // pooled-key moments (Gaussian threshold)
   w.theta = w.kmom + align_up(bh * (d + static_cast<size_t>(d) * d) * sizeof(float), kAlign);
-  w.total = w.theta + align_up(bh * nblocks(N, Bq) * sizeof(float), kAlign);
+  w.kbar16 = w.theta + align_up(bh * nblocks(N, Bq) * sizeof(float), kAlign);  // token-to-block correction
+  w.vbar16 = w.kbar16 + align_up(bh * nblocks(N, Bk) * d * 2, kAlign);
+  w.total = w.vbar16 + align_up(bh * nblocks(N, Bk) * d * 2, kAlign);
   return w;
 }
 
@@ -122,30 +124,39 @@ int launch_pool(const PoolArgs &args, int BH, int d, int max_nb, cudaStream_t st
   return cudaGetLastError() == cudaSuccess ? SOLATTN_OK : SOLATTN_ECUDA;
 }
 
-template <class C>
-int launch_fwd(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv, const FwdParams &p, int sms,
-               cudaStream_t st) {
+template <class C, bool TOKEN>
+int launch_fwd_v(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv, const CUtensorMap &mkp,
+                 const CUtensorMap &mvp, const FwdParams &p, int sms, cudaStream_t st) {
   constexpr size_t smem = fwd_smem_bytes<C>();
   static bool attr_set[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64) return SOLATTN_ECUDA;
   if (!attr_set[dev]) {
-    if (cudaFuncSetAttribute(solattn_fwd_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(solattn_fwd_kernel<C, TOKEN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)
       return SOLATTN_ECUDA;
     attr_set[dev] = true;
   }
   const int grid = p.n_items < sms ? p.n_items : sms;
-  solattn_fwd_kernel<C><<<grid, C::NUM_THREADS, smem, st>>>(mq, mk, mv, p);
+  solattn_fwd_kernel<C, TOKEN><<<grid, C::NUM_THREADS, smem, st>>>(mq, mk, mv, mkp, mvp, p);
   return cudaGetLastError() == cudaSuccess ? SOLATTN_OK : SOLATTN_ECUDA;
 }
 
+// The kernel with pseudo-tile handling only when the token-to-block correction is on.
+template <class C>
+int launch_fwd(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv, const CUtensorMap &mkp,
+               const CUtensorMap &mvp, const FwdParams &p, int sms, cudaStream_t st) {
+  return p.token_corr ? launch_fwd_v<C, true>(mq, mk, mv, mkp, mvp, p, sms, st)
+                      : launch_fwd_v<C, false>(mq, mk, mv, mkp, mvp, p, sms, st);
+}
+
 template <int D, int BK, int SUBQ>
-int dispatch_tiles(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv, FwdParams p, int sms,
+int dispatch_tiles(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv, const CUtensorMap &mkp,
+                   const CUtensorMap &mvp, FwdParams p, int sms,
                    cudaStream_t st) {
   using C = Cfg<D, BK, SUBQ>;
-  return launch_fwd<C>(mq, mk, mv, p, sms, st);
+  return launch_fwd<C>(mq, mk, mv, mkp, mvp, p, sms, st);
 }
 
 template <int D, int BK, int SUBQ>
@@ -171,18 +182,18 @@ int dispatch_plan(int d, int Bq, int Bk, const FwdParams &p, int *cost, int *ord
 }
 
 int dispatch(int d, int Bq, int Bk, const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
-             const FwdParams &p, int sms, cudaStream_t st) {
+             const CUtensorMap &mkp, const CUtensorMap &mvp, const FwdParams &p, int sms, cudaStream_t st) {
   const int subq = 128 / Bq;
   if (d == 128) {
-    if (Bk == 128) return subq == 1 ? dispatch_tiles<128, 128, 1>(mq, mk, mv, p, sms, st)
-                                    : dispatch_tiles<128, 128, 2>(mq, mk, mv, p, sms, st);
-    return subq == 1 ? dispatch_tiles<128, 64, 1>(mq, mk, mv, p, sms, st)
-                     : dispatch_tiles<128, 64, 2>(mq, mk, mv, p, sms, st);
+    if (Bk == 128) return subq == 1 ? dispatch_tiles<128, 128, 1>(mq, mk, mv, mkp, mvp, p, sms, st)
+                                    : dispatch_tiles<128, 128, 2>(mq, mk, mv, mkp, mvp, p, sms, st);
+    return subq == 1 ? dispatch_tiles<128, 64, 1>(mq, mk, mv, mkp, mvp, p, sms, st)
+                     : dispatch_tiles<128, 64, 2>(mq, mk, mv, mkp, mvp, p, sms, st);
   }
-  if (Bk == 128) return subq == 1 ? dispatch_tiles<64, 128, 1>(mq, mk, mv, p, sms, st)
-                                  : dispatch_tiles<64, 128, 2>(mq, mk, mv, p, sms, st);
-  return subq == 1 ? dispatch_tiles<64, 64, 1>(mq, mk, mv, p, sms, st)
-                   : dispatch_tiles<64, 64, 2>(mq, mk, mv, p, sms, st);
+  if (Bk == 128) return subq == 1 ? dispatch_tiles<64, 128, 1>(mq, mk, mv, mkp, mvp, p, sms, st)
+                                  : dispatch_tiles<64, 128, 2>(mq, mk, mv, mkp, mvp, p, sms, st);
+  return subq == 1 ? dispatch_tiles<64, 64, 1>(mq, mk, mv, mkp, mvp, p, sms, st)
+                   : dispatch_tiles<64, 64, 2>(mq, mk, mv, mkp, mvp, p, sms, st);
 }
 
 // ---- scratch for solattn_forward_noalloc
@@ -242,7 +253,7 @@ enum Rule { kRunningMax = 0, kGaussExact = 1, kGaussDiag = 2 };
 int forward_impl(const void *q, const void *k, const void *v, void *out, int B, int H, int N, int d, int Bq, int Bk,
                  float tau, int mode, const solattn_stats *stats, void *workspace, size_t ws_bytes, void *stream,
                  void *ev_attn_begin, void *ev_attn_end, int rule = kRunningMax, float beta = 0.f,
-                 int n_sink = 0) {
+                 int n_sink = 0, int token_corr = 0) {
   if (!q || !k || !v || !out || !stats || !stats->kept_per_head) return SOLATTN_EINVAL;
   const int rc = check_shape(B, H, N, d, Bq, Bk);
   if (rc != SOLATTN_OK) return rc;
@@ -253,6 +264,8 @@ int forward_impl(const void *q, const void *k, const void *v, void *out, int B, 
     return SOLATTN_EINVAL;  // NaN
   }
   if (n_sink < 0 || n_sink > N) return SOLATTN_EINVAL;
+  if (token_corr != 0 && token_corr != 1) return SOLATTN_EINVAL;
+  const bool token = token_corr && mode == SOLATTN_KEEP_CORRECT;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16)) return SOLATTN_EINVAL;
   if (!aligned(stats->kept_per_head, 8) || (stats->keep_mask && !aligned(stats->keep_mask, 4)))
     return SOLATTN_EINVAL;
@@ -271,10 +284,22 @@ int forward_impl(const void *q, const void *k, const void *v, void *out, int B, 
   float *vbar = reinterpret_cast<float *>(ws + wl.vbar);
   __half *v16 = reinterpret_cast<__half *>(ws + wl.v16);
 
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mq, mk, mv, mkp, mvp;
   if (make_map(&mq, q, d, N, BH, 128) != SOLATTN_OK || make_map(&mk, k, d, N, BH, Bk) != SOLATTN_OK ||
       make_map(&mv, v16, d, N, BH, Bk, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) != SOLATTN_OK)
     return SOLATTN_ECUDA;
+  // Token-to-block correction: the pooled keys (bf16) and values (fp16) of every head, read
+  // by the attention kernel as BK-row tiles; otherwise the K/V maps stand in (never read).
+  __nv_bfloat16 *kbar16 = reinterpret_cast<__nv_bfloat16 *>(ws + wl.kbar16);
+  __half *vbar16 = reinterpret_cast<__half *>(ws + wl.vbar16);
+  if (token) {
+    if (make_map(&mkp, kbar16, d, nKB, BH, Bk) != SOLATTN_OK ||
+        make_map(&mvp, vbar16, d, nKB, BH, Bk, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) != SOLATTN_OK)
+      return SOLATTN_ECUDA;
+  } else {
+    mkp = mk;
+    mvp = mv;
+  }
 
   if (cudaMemsetAsync(ws, 0, kHeaderBytes, st) != cudaSuccess) return SOLATTN_ECUDA;
   if (cudaMemsetAsync(stats->kept_per_head, 0, sizeof(int64_t) * BH, st) != cudaSuccess) return SOLATTN_ECUDA;
@@ -297,6 +322,12 @@ int forward_impl(const void *q, const void *k, const void *v, void *out, int B, 
     const int rcp = launch_pool(a, BH, d, nQB > nKB ? nQB : nKB, st);
     if (rcp != SOLATTN_OK) return rcp;
   }
+  if (token) {
+    const size_t n = static_cast<size_t>(BH) * nKB * d;
+    const int blocks = static_cast<int>((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);
+    pooled_copy_kernel<<<blocks, 256, 0, st>>>(kbar, vbar, kbar16, vbar16, n);
+    if (cudaGetLastError() != cudaSuccess) return SOLATTN_ECUDA;
+  }
 
   FwdParams p{};
   p.N = N;
@@ -318,6 +349,8 @@ int forward_impl(const void *q, const void *k, const void *v, void *out, int B, 
   p.order = nullptr;
   p.theta = nullptr;
   p.n_sink_blocks = nblocks(n_sink, Bk);
+  p.token_corr = token ? 1 : 0;
+  p.n_pseudo = token ? nblocks(nKB, Bk) : 0;
   if (mode != SOLATTN_DENSE && rule != kRunningMax) {
     float *kmom = reinterpret_cast<float *>(ws + wl.kmom);
     float *theta = reinterpret_cast<float *>(ws + wl.theta);
@@ -340,7 +373,7 @@ int forward_impl(const void *q, const void *k, const void *v, void *out, int B, 
   }
   if (ev_attn_begin && cudaEventRecord(static_cast<cudaEvent_t>(ev_attn_begin), st) != cudaSuccess)
     return SOLATTN_ECUDA;
-  const int rl = dispatch(d, Bq, Bk, mq, mk, mv, p, di.sms, st);
+  const int rl = dispatch(d, Bq, Bk, mq, mk, mv, mkp, mvp, p, di.sms, st);
   if (rl != SOLATTN_OK) return rl;
   if (ev_attn_end && cudaEventRecord(static_cast<cudaEvent_t>(ev_attn_end), st) != cudaSuccess)
     return SOLATTN_ECUDA;
@@ -419,7 +452,7 @@ int solattn_forward_ex(const void *q, const void *k, const void *v, void *out, i
     default: return SOLATTN_EINVAL;
   }
   return forward_impl(q, k, v, out, B, H, N, d, Bq, Bk, route->tau, mode, stats, workspace, ws_bytes, stream, nullptr,
-                      nullptr, rule, route->beta, route->n_sink);
+                      nullptr, rule, route->beta, route->n_sink, route->correction);
 }
 
 int solattn_get_status(const void *workspace, void *stream) {

@@ -33,6 +33,7 @@ EXPORTS = ("solattn_workspace_size", "solattn_pool", "solattn_forward", "solattn
            "solattn_strerror")
 GAUSS_VARIANTS = {"exact": 0, "diag": 1}  # solattn_gauss_variant
 RULES = {"running_max": 0, "gauss_exact": 1, "gauss_diag": 2}  # solattn_rule
+CORRECTIONS = {"block": 0, "token": 1}  # solattn_correction
 
 
 class SolAttnError(RuntimeError):
@@ -46,7 +47,8 @@ class _Stats(ctypes.Structure):
 
 
 class _Route(ctypes.Structure):  # solattn_route
-    _fields_ = [("rule", ctypes.c_int), ("tau", ctypes.c_float), ("beta", ctypes.c_float), ("n_sink", ctypes.c_int)]
+    _fields_ = [("rule", ctypes.c_int), ("tau", ctypes.c_float), ("beta", ctypes.c_float), ("n_sink", ctypes.c_int),
+                ("correction", ctypes.c_int)]
 
 
 def _load():
@@ -220,16 +222,20 @@ def solattn_forward_gaussian(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, 
 
 def solattn_forward_ex(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, Bq: int, Bk: int, mode="keep_correct",
                        rule="running_max", tau: float = 0.0, beta: float = 0.0, n_sink: int = 0,
-                       out: torch.Tensor | None = None, kept_per_head: torch.Tensor | None = None,
+                       correction="block", out: torch.Tensor | None = None,
+                       kept_per_head: torch.Tensor | None = None,
                        keep_mask: bool | torch.Tensor = False, workspace: torch.Tensor | None = None, stream=None):
     """The forward operator with every routing option: ``rule`` "running_max" (tau),
-    "gauss_exact" or "gauss_diag" (beta), and ``n_sink`` leading key tokens kept as sinks.
+    "gauss_exact" or "gauss_diag" (beta), ``n_sink`` leading key tokens kept as sinks, and
+    the keep_correct ``correction``: "block" (block proxy) or "token" (token-to-block logit).
     Returns what :func:`solattn_forward` returns."""
     if rule not in RULES:
         raise ValueError(f"unknown rule {rule!r}")
+    if correction not in CORRECTIONS:
+        raise ValueError(f"unknown correction {correction!r}")
     B, H, N, d, out, kept_per_head, mask, workspace, stats = _prepare(q, k, v, Bq, Bk, out, kept_per_head,
                                                                       keep_mask, workspace)
-    route = _Route(RULES[rule], float(tau), float(beta), int(n_sink))
+    route = _Route(RULES[rule], float(tau), float(beta), int(n_sink), CORRECTIONS[correction])
     rc = _lib.solattn_forward_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, H, N, d, Bq, Bk,
                                  ctypes.byref(route), _mode(mode), ctypes.byref(stats), workspace.data_ptr(),
                                  workspace.numel(), _stream(stream))

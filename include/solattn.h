@@ -214,7 +214,14 @@ typedef struct {
   float tau;   /* running-max rule: tau >= 0 (+infinity keeps every block)              */
   float beta;  /* Gaussian rules: standardized offset (not NaN; +-infinity allowed)     */
   int n_sink;  /* leading key tokens kept as sinks: 0 <= n_sink <= N                    */
+  int correction; /* keep_correct only: SOLATTN_CORR_BLOCK (0) or SOLATTN_CORR_TOKEN (1)   */
 } solattn_route;
+
+/* Correction of solattn_forward_ex in keep_correct mode. */
+typedef enum {
+  SOLATTN_CORR_BLOCK = 0,  /* dropped block j enters query block i with the block proxy s_ij     */
+  SOLATTN_CORR_TOKEN = 1   /* it enters row r with the token-to-block logit q_r . k_j / sqrt(d)   */
+} solattn_correction;
 
 /*
  * The forward operator with every routing option. Sinks: the text key-value tokens that
@@ -226,10 +233,17 @@ typedef struct {
  * and is never folded into the correction. The proxies of sink blocks still enter the
  * running maximum, so the other keep decisions do not change; under a Gaussian rule the
  * top-block guard applies only to a query block that would otherwise keep nothing.
- * With n_sink = 0, rule RUNNING_MAX equals solattn_forward and the Gaussian rules equal
- * solattn_forward_gaussian.
- * Errors: route NULL, an unknown rule, tau < 0 or NaN (running max), beta NaN (Gaussian)
- * or n_sink outside [0, N] -> SOLATTN_EINVAL; otherwise as solattn_forward.
+ * Token-to-block correction (keep_correct, correction = SOLATTN_CORR_TOKEN): the pages
+ * fuse routing and correction through a token-to-block score tile ("Unified execution",
+ * paperlayer summary §3). Each row r then meets every block j its query block dropped as
+ * one pseudo-key: logit q_r . k_j / sqrt(d) (pooled key k_j), weight n_j, value v_j,
+ * inside the same online softmax as the exact blocks (computed on the tensor cores over
+ * the head's pooled keys, with the kept blocks masked out).
+ * With n_sink = 0 and the block correction, rule RUNNING_MAX equals solattn_forward and
+ * the Gaussian rules equal solattn_forward_gaussian.
+ * Errors: route NULL, an unknown rule, tau < 0 or NaN (running max), beta NaN (Gaussian),
+ * n_sink outside [0, N] or an unknown correction -> SOLATTN_EINVAL; otherwise as
+ * solattn_forward.
  */
 int solattn_forward_ex(const void *q, const void *k, const void *v, void *out,
                        int B, int H, int N, int d, int Bq, int Bk, const solattn_route *route,

@@ -31,18 +31,18 @@ def unpack_mask(mask: torch.Tensor, nKB: int) -> np.ndarray:
     return bits[..., :nKB].astype(bool)
 
 
-def run_gpu(q, k, v, Bq, Bk, tau, mode, gauss=None, n_sink=0):
+def run_gpu(q, k, v, Bq, Bk, tau, mode, gauss=None, n_sink=0, correction="block"):
     """gauss: None (running-max rule with tau) or (beta, variant) for the Gaussian threshold;
-    n_sink > 0 goes through solattn_forward_ex."""
+    n_sink > 0 or the token correction go through solattn_forward_ex."""
     from block_sparse_online_b200 import solattn
     dev = torch.device("cuda:0")
     qd, kd, vd = (t.to(dev).contiguous() for t in (q, k, v))
     ws = solattn.alloc_workspace(*qd.shape, Bq, Bk, dev)
-    if n_sink:
+    if n_sink or correction != "block":
         rule = "running_max" if gauss is None else f"gauss_{gauss[1]}"
         out, kept, mask = solattn.solattn_forward_ex(qd, kd, vd, Bq, Bk, mode, rule, tau=tau,
                                                      beta=0.0 if gauss is None else gauss[0], n_sink=n_sink,
-                                                     keep_mask=True, workspace=ws)
+                                                     correction=correction, keep_mask=True, workspace=ws)
     elif gauss is None:
         out, kept, mask = solattn.solattn_forward(qd, kd, vd, Bq, Bk, tau, mode, keep_mask=True, workspace=ws)
     else:
@@ -54,13 +54,13 @@ def run_gpu(q, k, v, Bq, Bk, tau, mode, gauss=None, n_sink=0):
     return out.cpu(), kept.cpu(), mask
 
 
-def check_case(q, k, v, Bq, Bk, tau, mode, qblocks=None, label="", gauss=None, n_sink=0):
+def check_case(q, k, v, Bq, Bk, tau, mode, qblocks=None, label="", gauss=None, n_sink=0, correction="block"):
     """Run one case on the GPU and compare keep sets, counts and outputs with the oracle.
     gauss: None (running-max rule with tau) or (beta, variant); n_sink: sink tokens.
     Returns a dict of the measured errors."""
     B, H, N, d = q.shape
     nQB, nKB = -(-N // Bq), -(-N // Bk)
-    out, kept, mask = run_gpu(q, k, v, Bq, Bk, tau, mode, gauss, n_sink)
+    out, kept, mask = run_gpu(q, k, v, Bq, Bk, tau, mode, gauss, n_sink, correction)
     gpu_keep = unpack_mask(mask, nKB)
     if gauss is None:
         ref_keep, margin, _ = ref.keep_sets(q, k, Bq, Bk, tau, mode, n_sink=n_sink)
@@ -75,7 +75,7 @@ def check_case(q, k, v, Bq, Bk, tau, mode, qblocks=None, label="", gauss=None, n
     np.testing.assert_array_equal(kept.numpy(), gpu_keep.sum(axis=(-1, -2)))
     if not flips:
         np.testing.assert_array_equal(kept.numpy(), ref.kept_per_head(ref_keep))
-    want, _ = ref.forward(q, k, v, Bq, Bk, tau, mode, keep=gpu_keep, qblocks=qblocks)
+    want, _ = ref.forward(q, k, v, Bq, Bk, tau, mode, keep=gpu_keep, qblocks=qblocks, correction=correction)
     got = out.to(torch.float64).numpy()
     sel = ~np.isnan(want[..., 0])
     w, g = want[sel], got[sel]

@@ -252,3 +252,51 @@ def test_forward_ex_without_sinks_matches_the_other_entry_points():
     torch.cuda.synchronize()
     assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
     assert torch.equal(c[0], e[0]) and torch.equal(c[1], e[1])
+
+
+# ------------------------------------------------------------ token-to-block correction
+
+TOKEN_SHAPES = [
+    (1, 2, 1000, 64, 64, 64),
+    (1, 2, 777, 128, 128, 64),
+    (2, 1, 1300, 128, 64, 128),
+    (1, 1, 50, 64, 64, 64),
+]
+
+
+@pytest.mark.parametrize("shape", TOKEN_SHAPES, ids=[str(s) for s in TOKEN_SHAPES])
+def test_token_correction_shapes(shape):
+    B, H, N, d, Bq, Bk = shape
+    cfg = synth.Config("adhoc", B=B, H=H, d=d, grid=(1, 1, N), Bq=Bq, Bk=Bk, taus=(), seed=51 + N)
+    q, k, v = synth.make_inputs(cfg)
+    for tau in (0.0, 1.5, 3.0):
+        check_case(q, k, v, Bq, Bk, tau, "keep_correct", correction="token", label=f"{shape} token {tau}")
+    check_case(q, k, v, Bq, Bk, 0.0, "keep_correct", gauss=(1.0, "exact"), n_sink=min(70, N), correction="token",
+               label=f"{shape} token gauss sinks")
+
+
+def test_token_correction_exact_for_block_constant_keys():
+    """K constant inside each key block: the token-to-block correction reproduces dense attention."""
+    g = torch.Generator().manual_seed(6)
+    N, d, blk = 1000, 128, 128
+    nb = -(-N // blk)
+    kb = torch.randn(nb, d, generator=g) * 0.6
+    k = kb.repeat_interleave(blk, 0)[:N].to(torch.bfloat16)[None, None].contiguous()
+    q = (torch.randn(1, 1, N, d, generator=g) * 0.8).to(torch.bfloat16)
+    v = torch.randn(1, 1, N, d, generator=g).to(torch.bfloat16)
+    dense, _, _ = run_gpu(q, k, v, blk, blk, 0.0, "dense")
+    for tau in (0.0, 0.02):  # the proxies here span about 0.14: these taus drop blocks
+        out, kept, mask = run_gpu(q, k, v, blk, blk, tau, "keep_correct", correction="token")
+        assert unpack_mask(mask, nb).mean() < 1.0
+        err = (out.double() - dense.double()).abs()
+        tol = 2e-3 + 2 * torch.from_numpy(half_ulp_bf16(dense.double().numpy()))
+        assert (err <= tol).all(), err.max().item()
+
+
+def test_token_correction_video480_config():
+    cfg = synth.CONFIGS["video480"]
+    q, k, v = synth.make_inputs(cfg)
+    blocks = sampled_blocks(cfg.B, cfg.H, cfg.N, cfg.Bq, cfg.Bk, 4, seed=cfg.seed)
+    for tau in (3.0, 6.0):
+        check_case(q, k, v, cfg.Bq, cfg.Bk, tau, "keep_correct", qblocks=blocks, correction="token",
+                   label=f"video480 token {tau}")

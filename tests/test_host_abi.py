@@ -127,13 +127,13 @@ def test_forward_gaussian_accepts_infinite_beta_and_negative_beta():
         assert _call_gauss(beta=beta) in (solattn.SOLATTN_ECUDA, solattn.SOLATTN_EUNSUPPORTED)
 
 
-def _call_ex(rule=0, tau=1.0, beta=0.0, n_sink=0, route=True, **kw):
+def _call_ex(rule=0, tau=1.0, beta=0.0, n_sink=0, route=True, correction=0, **kw):
     """solattn_forward_ex with placeholder pointers (invalid cases only, as _call)."""
     a = dict(q=4096, k=4096, v=4096, out=4096, B=1, H=1, N=256, d=128, Bq=128, Bk=128, mode=2, kept=4096,
              mask=None, ws=4096, ws_bytes=1 << 30)
     a.update(kw)
     st = solattn._Stats(a["kept"], a["mask"])
-    r = solattn._Route(rule, tau, beta, n_sink)
+    r = solattn._Route(rule, tau, beta, n_sink, correction)
     return solattn._lib.solattn_forward_ex(a["q"], a["k"], a["v"], a["out"], a["B"], a["H"], a["N"], a["d"],
                                            a["Bq"], a["Bk"], ctypes.byref(r) if route else None, a["mode"],
                                            ctypes.byref(st), a["ws"], a["ws_bytes"], None)
@@ -147,6 +147,7 @@ def _call_ex(rule=0, tau=1.0, beta=0.0, n_sink=0, route=True, **kw):
     (dict(rule=1, beta=float("nan")), solattn.SOLATTN_EINVAL),
     (dict(n_sink=-1), solattn.SOLATTN_EINVAL),
     (dict(n_sink=257), solattn.SOLATTN_EINVAL),   # more sinks than key tokens
+    (dict(correction=2), solattn.SOLATTN_EINVAL),
     (dict(q=None), solattn.SOLATTN_EINVAL),
 ])
 def test_forward_ex_rejects_bad_arguments(kw, want):
@@ -157,7 +158,8 @@ def test_forward_ex_rejects_bad_arguments(kw, want):
 def test_forward_ex_accepts_valid_routes():
     # Valid options (a negative tau is valid under a Gaussian rule, n_sink = N is valid);
     # without a GPU the call fails only at the device query.
-    for kw in (dict(rule=1, tau=-1.0, beta=1.0), dict(rule=2, n_sink=256), dict(rule=0, tau=float("inf"))):
+    for kw in (dict(rule=1, tau=-1.0, beta=1.0), dict(rule=2, n_sink=256), dict(rule=0, tau=float("inf")),
+               dict(correction=1)):
         assert _call_ex(**kw) in (solattn.SOLATTN_ECUDA, solattn.SOLATTN_EUNSUPPORTED)
 
 
