@@ -239,6 +239,20 @@ def dist_setup(args):
     return world, rank, local
 
 
+METRIC = "sparse-attn dense-equiv TFLOP/s (ms/call, executed TFLOP/s and keep ratio alongside)"
+UNIT = "TFLOP/s (dense-equivalent)"
+
+
+def config_dict(args, cfg, world):
+    """The workload description both arms print."""
+    B, H, N, d = cfg.shape()
+    elem = B * H * N * d
+    return {"workload": f"{args.config}: {cfg.note}", "mode": args.mode, "tau": args.tau,
+            "B": B, "H": H, "N": N, "d": d, "Bq": cfg.Bq, "Bk": cfg.Bk,
+            "l2": "inputs larger than L2 (q, k, v = %.0f MB)" % (3 * elem * 2 / 1e6),
+            "parallelism": f"replicas x{world}"}
+
+
 def reference_arm(args, world, rank):
     if rank != 0:
         return
@@ -253,14 +267,14 @@ def reference_arm(args, world, rank):
             vals.append(rate)
     value = statistics.median(vals)
     line = {
-        "impl": "reference", "metric": "sparse-attn dense-equiv TFLOP/s (fp64 CPU oracle)", "value": value,
-        "unit": "TFLOP/s (dense-equivalent)", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "impl": "reference", "metric": METRIC, "value": value,
+        "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": cfg.dense_flops() / (value * 1e12) * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": f"{args.config}: {cfg.note}", "tau": args.tau, "mode": args.mode},
-        "cpu_baseline": {"value": value, "unit": "TFLOP/s (dense-equivalent)", "cores": cores(), "kind": "oracle",
+        "config": config_dict(args, cfg, world),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores(), "kind": "oracle",
                          "sample": desc},
-        "e2e": {"value": value, "unit": "TFLOP/s (dense-equivalent)", "h2d_bytes_per_step": 0,
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -466,14 +480,11 @@ def main():
 
     if rank == 0:
         line = {
-            "metric": "sparse-attn dense-equiv TFLOP/s (ms/call, executed TFLOP/s and keep ratio alongside)",
-            "value": round(value, 3), "unit": "TFLOP/s (dense-equivalent)", "n_gpus": world, "steps": args.steps,
+            "metric": METRIC,
+            "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": f"{args.config}: {cfg.note}", "mode": args.mode, "tau": args.tau,
-                       "B": B, "H": H, "N": N, "d": d, "Bq": cfg.Bq, "Bk": cfg.Bk,
-                       "l2": "inputs larger than L2 (q, k, v = %.0f MB)" % (3 * elem * 2 / 1e6),
-                       "parallelism": f"replicas x{world}"},
+            "config": config_dict(args, cfg, world),
             "keep_ratio": round(float(bits.mean()), 5),
             "exec_tflops": round(exec_flops / (ms_step * 1e-3) / 1e12, 2),
             "step_ms_median": round(statistics.median(step_ms), 4),
