@@ -24,6 +24,9 @@
  *                  keep_drop:    the same without the dropped terms
  *                  dense:        every block kept (plain softmax attention)
  *   with s_rc = q_r . k_c / sqrt(d).
+ * These are the definitions of solattn_forward. solattn_forward_gaussian and
+ * solattn_forward_ex add the pages' query-dependent Gaussian threshold, sink tokens and
+ * the token-to-block correction; each is defined where it is declared below.
  *
  * Data layout: q, k, v and out are contiguous row-major bf16 [B][H][N][d]
  * (token index n = (t*Y + y)*X + x for a (t, y, x) patch grid, t-major).
