@@ -128,15 +128,17 @@ template <class C, bool TOKEN>
 int launch_fwd_v(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv, const CUtensorMap &mkp,
                  const CUtensorMap &mvp, const FwdParams &p, int sms, cudaStream_t st) {
   constexpr size_t smem = fwd_smem_bytes<C>();
-  static bool attr_set[64] = {};
+  static bool attr_set[64] = {};  // per device; guarded by g_mu (calls may come from several threads)
   int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 0 || dev >= 64) return SOLATTN_ECUDA;
-  if (!attr_set[dev]) {
-    if (cudaFuncSetAttribute(solattn_fwd_kernel<C, TOKEN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem)) != cudaSuccess)
-      return SOLATTN_ECUDA;
-    attr_set[dev] = true;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return SOLATTN_ECUDA;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!attr_set[dev]) {
+      if (cudaFuncSetAttribute(solattn_fwd_kernel<C, TOKEN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(smem)) != cudaSuccess)
+        return SOLATTN_ECUDA;
+      attr_set[dev] = true;
+    }
   }
   const int grid = p.n_items < sms ? p.n_items : sms;
   solattn_fwd_kernel<C, TOKEN><<<grid, C::NUM_THREADS, smem, st>>>(mq, mk, mv, mkp, mvp, p);
@@ -241,6 +243,18 @@ int launch_threshold(int d, const float *qbar, const float *kbar, float *kmom, f
                  : launch_threshold_d<128>(qbar, kbar, kmom, theta, BH, nQB, nKB, beta, diag, st);
 }
 
+// A device pointer that belongs to another GPU than the current one (the kernels would
+// read or write it from the wrong device). Host, managed and unregistered pointers pass:
+// the alignment and null checks above cover them, and managed memory is reachable.
+bool foreign_device_pointer(const void *p, int dev) {
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    cudaGetLastError();  // clear the sticky-free error of an unknown pointer
+    return false;
+  }
+  return a.type == cudaMemoryTypeDevice && a.device != dev;
+}
+
 int items_total(int B, int H, int N) {
   // One work item per 128-row query tile.
   return B * H * ((N + 127) / 128);
@@ -274,6 +288,13 @@ int forward_impl(const void *q, const void *k, const void *v, void *out, int B, 
   DeviceInfo di;
   if (device_info(&di) != SOLATTN_OK) return SOLATTN_ECUDA;
   if (di.major != 10) return SOLATTN_EUNSUPPORTED;
+  {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return SOLATTN_ECUDA;
+    const void *ptrs[] = {q, k, v, out, stats->kept_per_head, stats->keep_mask, workspace};
+    for (const void *ptr : ptrs)
+      if (ptr && foreign_device_pointer(ptr, dev)) return SOLATTN_EINVAL;
+  }
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint8_t *ws = static_cast<uint8_t *>(workspace);

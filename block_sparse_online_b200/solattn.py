@@ -104,10 +104,32 @@ def _check(status: int, what: str):
         raise SolAttnError(status, what)
 
 
-def _stream(stream):
+def _stream(stream, device=None):
+    """The CUDA stream handle to pass to the library: ``stream``, or the current stream
+    of ``device`` (the tensors' device). A stream on another device is refused, since the
+    library launches on the current device."""
     if stream is None:
-        stream = torch.cuda.current_stream()
+        stream = torch.cuda.current_stream(device)
+    elif device is not None and stream.device != torch.device(device):
+        raise ValueError(f"stream is on {stream.device}, the tensors on {device}")
     return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check_buffer(t, name, dtypes, numel, device):
+    """A caller-provided buffer the library writes or reads through a raw pointer: it must
+    be contiguous, of an accepted dtype, hold at least ``numel`` elements and live on the
+    inputs' device (the library checks none of this; a short or foreign buffer would be
+    written out of bounds)."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype not in dtypes:
+        raise ValueError(f"{name} must have dtype {' or '.join(str(d) for d in dtypes)}, not {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if t.numel() < numel:
+        raise ValueError(f"{name} holds {t.numel()} elements, {numel} needed")
+    if t.device != torch.device(device):
+        raise ValueError(f"{name} is on {t.device}, the inputs on {device}")
 
 
 def _mode(mode) -> int:
@@ -143,29 +165,43 @@ def solattn_pool(x: torch.Tensor, blk: int, out: torch.Tensor | None = None, str
     nb = -(-N // blk)
     if out is None:
         out = torch.empty((B, H, nb, d), dtype=torch.float32, device=x.device)
-    _check(_lib.solattn_pool(x.data_ptr(), out.data_ptr(), B, H, N, d, blk, _stream(stream)), "solattn_pool")
+    _check_buffer(out, "out", (torch.float32,), B * H * nb * d, x.device)
+    with torch.cuda.device(x.device):
+        rc = _lib.solattn_pool(x.data_ptr(), out.data_ptr(), B, H, N, d, blk, _stream(stream, x.device))
+    _check(rc, "solattn_pool")
     return out
 
 
-def _prepare(q, k, v, Bq, Bk, out, kept_per_head, keep_mask, workspace):
-    """Checks the inputs and allocates what the caller did not pass."""
+def _inputs(q, k, v):
     B, H, N, d = _bhnd(q)
     for t in (q, k, v):
         if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous() or tuple(t.shape) != (B, H, N, d):
             raise ValueError("q, k, v must be contiguous bf16 CUDA tensors of one shape")
+        if t.device != q.device:
+            raise ValueError("q, k, v must be on one device")
+    return B, H, N, d
+
+
+def _prepare(q, k, v, Bq, Bk, out, kept_per_head, keep_mask, workspace):
+    """Checks the inputs and the buffers the caller passed, and allocates the others."""
+    B, H, N, d = _inputs(q, k, v)
     dev = q.device
     if out is None:
         out = torch.empty_like(q)
+    _check_buffer(out, "out", (torch.bfloat16,), B * H * N * d, dev)
     if kept_per_head is None:
         kept_per_head = torch.empty((B, H), dtype=torch.int64, device=dev)
+    _check_buffer(kept_per_head, "kept_per_head", (torch.int64,), B * H, dev)
     mask = None
+    nq, nk = -(-N // Bq), -(-N // Bk)
     if isinstance(keep_mask, torch.Tensor):
         mask = keep_mask
+        _check_buffer(mask, "keep_mask", (torch.int32, torch.uint32), B * H * nq * (-(-nk // 32)), dev)
     elif keep_mask:
-        nq, nk = -(-N // Bq), -(-N // Bk)
         mask = torch.empty((B, H, nq, -(-nk // 32)), dtype=torch.int32, device=dev)
     if workspace is None:
         workspace = alloc_workspace(B, H, N, d, Bq, Bk, dev)
+    _check_buffer(workspace, "workspace", (torch.uint8, torch.int8), 0, dev)
     stats = _Stats(kept_per_head.data_ptr(), mask.data_ptr() if mask is not None else None)
     return B, H, N, d, out, kept_per_head, mask, workspace, stats
 
@@ -185,18 +221,19 @@ def solattn_forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, Bq: int, 
     """
     B, H, N, d, out, kept_per_head, mask, workspace, stats = _prepare(q, k, v, Bq, Bk, out, kept_per_head,
                                                                       keep_mask, workspace)
-    args = (q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, H, N, d, Bq, Bk,
-            ctypes.c_float(float(tau)), _mode(mode), ctypes.byref(stats), workspace.data_ptr(),
-            workspace.numel(), _stream(stream))
-    if events is None:
-        rc = _lib.solattn_forward(*args)
-    else:
-        st = stream if stream is not None else torch.cuda.current_stream()
-        for e in events:
-            if e.cuda_event == 0:  # torch creates the CUDA event on its first record
-                e.record(st)
-        rc = _lib.solattn_forward_events(*args, ctypes.c_void_p(events[0].cuda_event),
-                                         ctypes.c_void_p(events[1].cuda_event))
+    with torch.cuda.device(q.device):
+        args = (q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, H, N, d, Bq, Bk,
+                ctypes.c_float(float(tau)), _mode(mode), ctypes.byref(stats), workspace.data_ptr(),
+                workspace.numel(), _stream(stream, q.device))
+        if events is None:
+            rc = _lib.solattn_forward(*args)
+        else:
+            st = stream if stream is not None else torch.cuda.current_stream(q.device)
+            for e in events:
+                if e.cuda_event == 0:  # torch creates the CUDA event on its first record
+                    e.record(st)
+            rc = _lib.solattn_forward_events(*args, ctypes.c_void_p(events[0].cuda_event),
+                                             ctypes.c_void_p(events[1].cuda_event))
     _check(rc, "solattn_forward")
     return out, kept_per_head, mask
 
@@ -212,10 +249,11 @@ def solattn_forward_gaussian(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, 
         raise ValueError(f"unknown variant {variant!r}")
     B, H, N, d, out, kept_per_head, mask, workspace, stats = _prepare(q, k, v, Bq, Bk, out, kept_per_head,
                                                                       keep_mask, workspace)
-    rc = _lib.solattn_forward_gaussian(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, H, N, d, Bq,
-                                       Bk, ctypes.c_float(float(beta)), GAUSS_VARIANTS[variant], _mode(mode),
-                                       ctypes.byref(stats), workspace.data_ptr(), workspace.numel(),
-                                       _stream(stream))
+    with torch.cuda.device(q.device):
+        rc = _lib.solattn_forward_gaussian(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, H, N, d,
+                                           Bq, Bk, ctypes.c_float(float(beta)), GAUSS_VARIANTS[variant],
+                                           _mode(mode), ctypes.byref(stats), workspace.data_ptr(),
+                                           workspace.numel(), _stream(stream, q.device))
     _check(rc, "solattn_forward_gaussian")
     return out, kept_per_head, mask
 
@@ -236,15 +274,19 @@ def solattn_forward_ex(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, Bq: in
     B, H, N, d, out, kept_per_head, mask, workspace, stats = _prepare(q, k, v, Bq, Bk, out, kept_per_head,
                                                                       keep_mask, workspace)
     route = _Route(RULES[rule], float(tau), float(beta), int(n_sink), CORRECTIONS[correction])
-    rc = _lib.solattn_forward_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, H, N, d, Bq, Bk,
-                                 ctypes.byref(route), _mode(mode), ctypes.byref(stats), workspace.data_ptr(),
-                                 workspace.numel(), _stream(stream))
+    with torch.cuda.device(q.device):
+        rc = _lib.solattn_forward_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, H, N, d, Bq, Bk,
+                                     ctypes.byref(route), _mode(mode), ctypes.byref(stats), workspace.data_ptr(),
+                                     workspace.numel(), _stream(stream, q.device))
     _check(rc, "solattn_forward_ex")
     return out, kept_per_head, mask
 
 
 def solattn_get_status(workspace: torch.Tensor, stream=None) -> int:
-    return int(_lib.solattn_get_status(workspace.data_ptr(), _stream(stream)))
+    if not workspace.is_cuda:
+        raise ValueError("workspace must be a CUDA tensor")
+    with torch.cuda.device(workspace.device):
+        return int(_lib.solattn_get_status(workspace.data_ptr(), _stream(stream, workspace.device)))
 
 
 def solattn_forward_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, Bq: int, Bk: int, tau: float,
@@ -256,18 +298,24 @@ def solattn_forward_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, Bq: 
     inside the library call, which returns after the stream is synchronised."""
     B, H, N, d = _bhnd(q)
     for t in (q, k, v):
-        if t.dtype != torch.bfloat16 or t.is_cuda or not t.is_contiguous():
-            raise ValueError("q, k, v must be contiguous bf16 host tensors")
+        if t.dtype != torch.bfloat16 or t.is_cuda or not t.is_contiguous() or tuple(t.shape) != (B, H, N, d):
+            raise ValueError("q, k, v must be contiguous bf16 host tensors of one shape")
     if out is None:
         out = torch.empty_like(q, pin_memory=True)
+    _check_buffer(out, "out", (torch.bfloat16,), B * H * N * d, "cpu")
     if kept_per_head is None:
         kept_per_head = torch.empty((B, H), dtype=torch.int64)
+    _check_buffer(kept_per_head, "kept_per_head", (torch.int64,), B * H, "cpu")
     need = solattn_host_workspace_size(B, H, N, d, Bq, Bk)
     if scratch is None:
         scratch = torch.empty(need, dtype=torch.uint8, device="cuda")
-    rc = _lib.solattn_forward_host(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, H, N, d, Bq, Bk,
-                                   ctypes.c_float(float(tau)), _mode(mode), kept_per_head.data_ptr(),
-                                   scratch.data_ptr(), scratch.numel(), _stream(stream))
+    if not scratch.is_cuda:
+        raise ValueError("scratch must be a CUDA tensor")
+    _check_buffer(scratch, "scratch", (torch.uint8, torch.int8), 0, scratch.device)
+    with torch.cuda.device(scratch.device):
+        rc = _lib.solattn_forward_host(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, H, N, d, Bq,
+                                       Bk, ctypes.c_float(float(tau)), _mode(mode), kept_per_head.data_ptr(),
+                                       scratch.data_ptr(), scratch.numel(), _stream(stream, scratch.device))
     _check(rc, "solattn_forward_host")
     return out, kept_per_head
 
@@ -276,8 +324,9 @@ def solattn_watchdog_selftest(limit_ns: int = 2_000_000, stream=None) -> int:
     """Run the device watchdog self-test; returns the status the kernel stored
     (SOLATTN_ETIMEOUT when a wait that nobody completes is abandoned on time)."""
     ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
-    _check(_lib.solattn_watchdog_selftest(ws.data_ptr(), ws.numel(), int(limit_ns), _stream(stream)),
-           "solattn_watchdog_selftest")
+    with torch.cuda.device(ws.device):
+        rc = _lib.solattn_watchdog_selftest(ws.data_ptr(), ws.numel(), int(limit_ns), _stream(stream, ws.device))
+    _check(rc, "solattn_watchdog_selftest")
     return solattn_get_status(ws, stream)
 
 
@@ -291,17 +340,18 @@ def solattn_forward_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, B
     (for callers that cannot allocate device memory). Output and count tensors are
     allocated here only when not given; the library call itself allocates nothing.
     Calls that overlap on the GPU race on the shared scratch."""
-    B, H, N, d = _bhnd(q)
-    for t in (q, k, v):
-        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous() or tuple(t.shape) != (B, H, N, d):
-            raise ValueError("q, k, v must be contiguous bf16 CUDA tensors of one shape")
+    B, H, N, d = _inputs(q, k, v)
     if out is None:
         out = torch.empty_like(q)
+    _check_buffer(out, "out", (torch.bfloat16,), B * H * N * d, q.device)
     if kept_per_head is None:
         kept_per_head = torch.empty((B, H), dtype=torch.int64, device=q.device)
+    _check_buffer(kept_per_head, "kept_per_head", (torch.int64,), B * H, q.device)
     stats = _Stats(kept_per_head.data_ptr(), None)
-    rc = _lib.solattn_forward_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, H, N, d, Bq, Bk,
-                                      ctypes.c_float(float(tau)), _mode(mode), ctypes.byref(stats), _stream(stream))
+    with torch.cuda.device(q.device):
+        rc = _lib.solattn_forward_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, H, N, d, Bq,
+                                          Bk, ctypes.c_float(float(tau)), _mode(mode), ctypes.byref(stats),
+                                          _stream(stream, q.device))
     _check(rc, "solattn_forward_noalloc")
     return out, kept_per_head
 
@@ -311,8 +361,9 @@ def solattn_selftest_exp2(x: torch.Tensor, stream=None) -> torch.Tensor:
     if x.dtype != torch.float32 or not x.is_cuda or not x.is_contiguous():
         raise ValueError("x must be a contiguous fp32 CUDA tensor")
     y = torch.empty_like(x)
-    _check(_lib.solattn_selftest_exp2(x.data_ptr(), y.data_ptr(), x.numel(), _stream(stream)),
-           "solattn_selftest_exp2")
+    with torch.cuda.device(x.device):
+        rc = _lib.solattn_selftest_exp2(x.data_ptr(), y.data_ptr(), x.numel(), _stream(stream, x.device))
+    _check(rc, "solattn_selftest_exp2")
     return y
 
 

@@ -38,7 +38,10 @@
  * solattn_forward_host, which synchronise the stream.
  *
  * Ownership: the caller allocates and owns every buffer (inputs, output,
- * statistics, workspace). The library keeps no allocation between calls.
+ * statistics, workspace). The library allocates nothing at run time. Its one
+ * device-memory holding is the static scratch of solattn_forward_noalloc
+ * (SOLATTN_NOALLOC_SCRATCH_BYTES), a module-scope device array that exists on
+ * every GPU where the library's module is loaded, for the life of the process.
  */
 #ifndef SOLATTN_H
 #define SOLATTN_H
@@ -60,7 +63,7 @@ typedef enum {
 /* Status codes. Argument errors are returned before any device work is queued. */
 typedef enum {
   SOLATTN_OK = 0,
-  SOLATTN_EINVAL = -1,       /* null pointer, misaligned pointer, N/B/H < 1, bad mode, tau < 0 or NaN */
+  SOLATTN_EINVAL = -1,       /* null, misaligned or other-GPU pointer, N/B/H < 1, bad mode, tau < 0 or NaN */
   SOLATTN_EUNSUPPORTED = -2, /* d or Bq/Bk not in {64,128}, nKB > 1024, B*H > 65535, no sm_100 device */
   SOLATTN_ECUDA = -3,        /* a CUDA runtime or driver call failed                          */
   SOLATTN_ETIMEOUT = -4,     /* a device-side wait ran past its limit (reported by get_status) */
@@ -120,6 +123,10 @@ int solattn_pool(const void *x, float *xbar, int B, int H, int N, int d, int blk
  *              must not be used by another call that runs at the same time
  *   stream     cudaStream_t (as void*)
  *
+ * Every device pointer must belong to the current device (cudaGetDevice): one that
+ * belongs to another GPU is rejected with SOLATTN_EINVAL. The buffers' sizes cannot be
+ * checked here; the caller guarantees the sizes stated above.
+ *
  * Returns SOLATTN_OK once the work is queued (errors inside the kernels are
  * reported by solattn_get_status), or an error code with nothing queued.
  */
@@ -158,8 +165,10 @@ int solattn_forward_events(const void *q, const void *k, const void *v, void *ou
  * allocator); its scratch is a static device array of SOLATTN_NOALLOC_SCRATCH_BYTES.
  *
  *   - The first call on a device looks up that array's device address
- *     (cudaGetSymbolAddress) with the device current; make this first call before
- *     any stream capture.
+ *     (cudaGetSymbolAddress) with the device current, and later calls on that device
+ *     reuse it; make this first call before any stream capture. cudaDeviceReset
+ *     unloads the module and may move the array: do not call this entry point on a
+ *     device after resetting it in the same process.
  *   - Shapes whose solattn_workspace_size(...) exceeds SOLATTN_NOALLOC_SCRATCH_BYTES
  *     are rejected with SOLATTN_EWORKSPACE before any device work.
  *   - Every call on a device uses the same scratch, which keeps the previous call's

@@ -366,14 +366,6 @@ def keep_sets_gaussian(q, k, Bq: int, Bk: int, beta: float, variant: str = "exac
     return keep, margin, sbar
 
 
-def forward_gaussian(q, k, v, Bq: int, Bk: int, beta: float, variant: str = "exact", mode="keep_correct",
-                     keep: np.ndarray | None = None, qblocks=None, n_sink: int = 0, correction: str = "block"):
-    """Output under the Gaussian threshold (steps 1, 2 and 5 as in ``forward``)."""
-    if keep is None:
-        keep, _, _ = keep_sets_gaussian(q, k, Bq, Bk, beta, variant, mode, n_sink)
-    return forward(q, k, v, Bq, Bk, 0.0, mode, keep=keep, qblocks=qblocks, correction=correction)
-
-
 def sample_qblocks(B, H, nQB, Bq, Bk, nKB, per_head=64, seed=0):
     """Seeded sample of query blocks per head, plus block 0, the last (ragged) one and
     the blocks whose diagonal is at the extremes."""

@@ -3,11 +3,12 @@ exponentials (Cody & Waite range reduction to f in [-1/2, 1/2] plus a cubic mini
 fit of 2^f): the cubic, evaluated by Horner in fp32 as the kernel does, stays within
 the stated relative error bound of 7.5e-5 on the reduced interval, and the bound is
 equioscillating (no systematic bias)."""
+import os
 import re
 
 import numpy as np
 
-from tests.test_host_abi import ROOT
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
 def coefficients():

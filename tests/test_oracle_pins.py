@@ -383,8 +383,42 @@ def pin_token_correction():
         np.testing.assert_allclose(out[:, :, rows], want, rtol=1e-9, atol=1e-10)
 
 
+def pin_kept_per_head():
+    """Per-head kept-block counts (the statistic the operator returns): the hand-worked case
+    keeps blocks {0} for query block 0 and {0, 1} for query block 1 at tau = 1, i.e. 3 for its
+    only head; on a ragged multi-head case the count equals a scalar loop over the keep
+    decisions taken one (b, h, i, j) at a time from the proxies and the visit order."""
+    g = json.load(open(GOLDEN))
+    env = {"ln4": math.log(4.0), "ln2": math.log(2.0), "sqrt2": math.sqrt(2.0)}
+    ev = lambda x: float(eval(str(x), {"__builtins__": {}}, env))  # closed forms only
+    q = np.array([[ev(x) for x in r] for r in g["q"]])[None, None]
+    k = np.array([[ev(x) for x in r] for r in g["k"]])[None, None]
+    keep, _, _ = ref.keep_sets(q, k, g["Bq"], g["Bk"], 1.0, "keep_drop")
+    counts = ref.kept_per_head(keep)
+    assert counts.shape == (1, 1) and counts.dtype == np.int64 and int(counts[0, 0]) == 3
+    B, H, N, d, Bq, Bk, tau = 2, 3, 205, 8, 32, 16, 0.7
+    q, k, _ = _rand(B, H, N, d, seed=21)
+    keep, _, sbar = ref.keep_sets(q, k, Bq, Bk, tau, "keep_correct")
+    nQB, nKB = -(-N // Bq), -(-N // Bk)
+    want = np.zeros((B, H), dtype=np.int64)
+    for b in range(B):
+        for h in range(H):
+            for i in range(nQB):
+                j0 = min(i * Bq // Bk, nKB - 1)
+                m = -math.inf
+                for t in range(nKB):
+                    j = (j0 + t) % nKB
+                    m = max(m, sbar[b, h, i, j])
+                    want[b, h] += int(sbar[b, h, i, j] >= m - tau)
+    got = ref.kept_per_head(keep)
+    assert got.shape == (B, H) and np.array_equal(got, want), (got, want)
+    # dense mode keeps every pair
+    dense, _, _ = ref.keep_sets(q, k, Bq, Bk, tau, "dense")
+    assert np.array_equal(ref.kept_per_head(dense), np.full((B, H), nQB * nKB))
+
+
 PINS += [pin_gaussian_matches_row_statistics, pin_gaussian_diagonal_design, pin_gaussian_keep_fraction,
-         pin_gaussian_limits_and_monotone, pin_sinks, pin_token_correction]
+         pin_gaussian_limits_and_monotone, pin_sinks, pin_token_correction, pin_kept_per_head]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
@@ -492,6 +526,14 @@ def _mut_token_no_multiplicity(q_rows, kbar, dropped, counts, vbar):
     return (q_rows @ kbar[idx].T) / math.sqrt(d), np.ones(idx.size), vbar[idx]
 
 
+def _mut_kept_counts_dropped(keep):
+    return (~keep).sum(axis=(-1, -2)).astype(np.int64)
+
+
+def _mut_kept_one_block_axis(keep):
+    return keep.sum(axis=-1)[..., 0].astype(np.int64)
+
+
 MUTANTS = {
     "pool divides by block size": ("pool", _mut_pool_by_blk),
     "proxy without 1/sqrt(d)": ("proxy", _mut_proxy_unscaled),
@@ -510,6 +552,8 @@ MUTANTS = {
     "sink blocks rounded down": ("sink_blocks", _mut_sink_blocks_floor),
     "token correction with the block logit": ("correction_terms_token", _mut_token_uses_block_logit),
     "token correction without n_j": ("correction_terms_token", _mut_token_no_multiplicity),
+    "kept count of the dropped blocks": ("kept_per_head", _mut_kept_counts_dropped),
+    "kept count of one query block only": ("kept_per_head", _mut_kept_one_block_axis),
 }
 
 
