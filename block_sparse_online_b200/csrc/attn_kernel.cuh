@@ -8,8 +8,9 @@
 //   warps 1, 3  MMA issuers (one thread each, for warpgroups A and B, taking turns):
 //               S = Q K_j^T into tensor memory (TMEM, bf16 -> fp32), O += P V_j with P
 //               read from TMEM (fp16 -> fp32).
-//   warp 2      router: on-the-fly block thresholding and the correction sums for the
-//               NEXT item (double-buffered), from the fp32 pooled blocks in L2.
+//   warp 2      router: on-the-fly block thresholding for the NEXT item (double-buffered),
+//               from the fp32 pooled blocks in L2; it picks up each query block's
+//               correction sums, which the planning pass folded (keep_correct).
 //   warps 4..7  softmax warpgroup A, warps 8..11 softmax warpgroup B. The tile's kept
 //               list is split between them (A takes entries 0, 2, 4, ..., B takes 1, 3,
 //               5, ...); each keeps its own S, O, running max and sum for all 128 rows.
@@ -32,7 +33,9 @@
 //  * each dropped block re-enters as one pseudo-key of weight n_j e^{s} and value
 //    mean(V_j) ("Approximate correction": zeroth-order proxy-score reuse with pooled
 //    keys and summed values). Because s does not depend on the query row, the
-//    correction is one d-vector and one scalar per query block, built by the router.
+//    correction is one d-vector and one scalar per query block. The planning pass
+//    (plan_kernel), which routes every query tile before this kernel, folds it with the
+//    whole GPU's parallelism; the router here only takes the keep decisions.
 #pragma once
 
 #include <cstdint>
@@ -57,10 +60,9 @@ constexpr float kLog2e = 1.4426950408889634f;
 // Lazy rescaling: a row's reference max moves only when the tile max exceeds it by
 // more than this many log2 units, so P stays <= 2^8 and O is rarely rescaled.
 constexpr float kRescaleSlack = 8.0f;
-// One pair of exponentials in this many is computed on the FMA pipe (polynomial)
-// instead of the MUFU unit. Measured against 3, 4, 6 and none in the same run: 8 is the
-// fastest (the polynomial's extra instructions cost issue slots the softmax also needs).
-constexpr int kPolyEvery = 8;
+// Pairs of exponentials computed on the FMA pipe (polynomial) instead of the MUFU unit:
+// bit e % 8 of this mask set -> pair e of a 16-pair chunk goes to the polynomial.
+constexpr uint32_t kPolyMask = 0x80u;
 
 struct FwdParams {
   int N;
@@ -91,7 +93,16 @@ struct FwdParams {
   // to the tensor cores as n_pseudo tiles of pooled keys at the end of every item.
   int token_corr;
   int n_pseudo;
+  // keep_correct with the block correction: per (b, h, query block), {M, L, -, -, C[D]}
+  // (corr_stride floats), written by plan_kernel and read by the router.
+  float *corr;
 };
+
+// Floats per query block of the correction record: M (running proxy max, natural-log
+// units), L = sum over dropped j of n_j e^{s_ij - M}, two pad words, then
+// C = sum over dropped j of n_j e^{s_ij - M} mean(V_j) (16-byte aligned).
+template <int D>
+__host__ __device__ constexpr int corr_stride() { return D + 4; }
 
 template <int D_, int BK_, int SUBQ_>
 struct Cfg {
@@ -117,10 +128,11 @@ struct Cfg {
   static constexpr int NUM_THREADS = 32 * CTRL_WARPS + 128 * NWG;
   // Register split: the control warpgroup hands registers to the softmax warpgroups.
   // The sum stays within the registers the block is launched with (384 threads x 168).
-  // The softmax streams S in 32-column chunks (about 100 live registers); the router and
-  // MMA issuers spill below about 150.
-  static constexpr int CTRL_REGS = 152;
-  static constexpr int SOFTMAX_REGS = 176;
+  // The softmax holds a whole row of S (BK fp32 values) in registers and needs about 190;
+  // the router and MMA issuers fit in 120 (ptxas -v: no spill beyond the 12 bytes of the
+  // kernel's stack in the headline instantiation).
+  static constexpr int CTRL_REGS = 120;
+  static constexpr int SOFTMAX_REGS = 192;
   static_assert(128 * CTRL_REGS + 256 * SOFTMAX_REGS <= 384 * 168, "register split");
   // S = Q K^T in bf16; O += P V in fp16 (P in [0, 2^8] after the lazy rescale; V is the
   // fp16 copy written by the pooling pass).
@@ -377,16 +389,27 @@ __device__ __forceinline__ int route_block(const FwdParams &p, int bh, int qb, i
 template <class C>
 __device__ __forceinline__ void route_query_block(SmemCtl<C> &sc, RouteSlot<C> &rs, const FwdParams &p,
                                                   int bh, int sb, int qb, int lane) {
-  constexpr int VPL = C::D / 32;
+  constexpr int D = C::D;
+  constexpr int VPL = D / 32;
   const bool correct = (p.mode == 2) && !p.token_corr;  // block-level correction sums
   float cacc[VPL];
   float lacc, M;
-  route_block<C::D, C::BQ, C::BK>(p, bh, qb, lane, correct, sc.mask[sb], cacc, lacc, M);
-#pragma unroll
-  for (int e = 0; e < VPL; ++e) rs.Cv[sb][lane * VPL + e] = correct ? cacc[e] : 0.f;
-  if (lane == 0) {
-    rs.L[sb] = correct ? lacc : 0.f;
-    rs.M[sb] = correct ? M : -CUDART_INF_F;
+  // Keep decisions only: the correction sums of this query block were folded by the
+  // planning pass, through the same route_scan and hence the same decisions.
+  route_block<C::D, C::BQ, C::BK>(p, bh, qb, lane, false, sc.mask[sb], cacc, lacc, M);
+  if (correct) {
+    const float *rec = p.corr + (static_cast<size_t>(bh) * p.nQB + qb) * corr_stride<D>();
+    for (int e = lane; e < D; e += 32) rs.Cv[sb][e] = __ldg(rec + 4 + e);
+    if (lane == 0) {
+      rs.M[sb] = __ldg(rec);
+      rs.L[sb] = __ldg(rec + 1);
+    }
+  } else {
+    for (int e = lane; e < D; e += 32) rs.Cv[sb][e] = 0.f;
+    if (lane == 0) {
+      rs.L[sb] = 0.f;
+      rs.M[sb] = -CUDART_INF_F;
+    }
   }
 }
 
@@ -679,17 +702,21 @@ __device__ void run_mma(SmemCtl<C> &sc, const FwdParams &p, uint32_t tmem, uint8
     }
     bool first = true;
     for (int u = w; u < n && ok; u += 2) {
+      // Everything the group needs except P is waited for first (V_u and K_{u+2} landed,
+      // O free), so that once the softmax hands over P only the turn remains. K_{u+2}'s ring
+      // slot is freed by S_w(u)'s completion and O by the previous item's epilogue, both
+      // independent of P_w(u).
       const int vs = slot_of(ring_index_v(u, n));
       if (vs < 0) break;
-      if (!wait(&sc.p_full[w], p_ph)) break;
-      p_ph ^= 1;
-      // The first P V of the item overwrites O: the previous item's epilogue must be done.
-      if (first && !wait(&sc.o_empty, (o_it & 1) ^ 1)) break;
       int ks = -1;
       if (u + 2 < n) {
         ks = slot_of(ring_index_k(u + 2, n));
         if (ks < 0) break;
       }
+      // The first P V of the item overwrites O: the previous item's epilogue must be done.
+      if (first && !wait(&sc.o_empty, (o_it & 1) ^ 1)) break;
+      if (!wait(&sc.p_full[w], p_ph)) break;
+      p_ph ^= 1;
       const uint32_t g = (n == 1) ? 1u : static_cast<uint32_t>(2 + u);
       if (!turn(g)) break;
       issue_pv<C>(tmem, w, v_desc0 + static_cast<uint64_t>(vs * kSlotUnits), !first);
@@ -833,44 +860,27 @@ __device__ void run_softmax(SmemCtl<C> &sc, const FwdParams &p, uint32_t tmem, i
       float alpha = 1.f;  // rescale of this row's O and l for this S tile
       float lsum = 0.f;
       if (!TOKEN || !(j & kPseudoFlag)) {
-        // Two passes over the row of S, 32 columns per TMEM load, each load issued one chunk
-        // ahead: the row maximum (a tree of three-input max instructions per chunk), then the
-        // exponentials, whose fp16 pairs go back to TMEM 16 columns at a time. The reference
-        // max only moves when the row maximum exceeds it by more than the slack (O and l are
-        // then rescaled once, below).
+        // One pass over the row of S held in registers: all BK columns are loaded at once
+        // (BK / 32 TMEM loads, one wait), the row maximum is a tree of three-input max
+        // instructions, and the exponentials go back to TMEM as fp16 pairs, 16 columns per
+        // store. The reference max only moves when the row maximum exceeds it by more than
+        // the slack (O and l are then rescaled once, below), so P never needs rescaling.
         constexpr int NCH = BK / 32;
         const bool rk = (mem & row_bit) != 0;  // warp-uniform (a warp's rows share a query block)
         const int ncol = (j == p.nKB - 1) ? (p.N - j * BK) : BK;
-        const bool full = rk && ncol == BK;    // no column of this block masked
         float mx = -CUDART_INF_F;
-        uint32_t x[32];
+        uint32_t x[BK];
         if (rk) {
-          tmem_ld32(s_addr, x);
+#pragma unroll
+          for (int c = 0; c < NCH; ++c) tmem_ld32(s_addr + c * 32, *reinterpret_cast<uint32_t(*)[32]>(x + c * 32));
           tmem_wait_ld();
-          reg_fence32(x);
-  #pragma unroll
-          for (int c = 0; c < NCH; ++c) {
-            uint32_t y[32];
-            // the next chunk, or (after the last) chunk 0 again for the exponential pass; the
-            // fence keeps the arithmetic on this chunk after the load is issued
-            tmem_ld32(s_addr + ((c + 1) % NCH) * 32, y);
-            reg_fence32(x);
-            float m;
-            if (full) {
-              m = max_tree_bits<32>(x);
-            } else {
-              m = -CUDART_INF_F;
-  #pragma unroll
-              for (int e = 0; e < 32; ++e)
-                if (c * 32 + e < ncol) m = fmaxf(m, u2f(x[e]));
-            }
-            mx = fmaxf(mx, m);
-            asm volatile("" ::"f"(mx));  // the tree stays ahead of the wait
-            tmem_wait_ld();
-            reg_fence32(y);
-  #pragma unroll
-            for (int e = 0; e < 32; ++e) x[e] = y[e];
+          reg_fence<BK>(x);
+          if (ncol < BK) {  // ragged last key block: columns past N are not keys
+#pragma unroll
+            for (int e = 0; e < BK; ++e)
+              if (e >= ncol) x[e] = __float_as_uint(-CUDART_INF_F);
           }
+          mx = max_tree_bits<BK>(x);
         }
         const float mxs = mx * sc_log2;
         if (mxs > m_ref + kRescaleSlack) {
@@ -878,64 +888,45 @@ __device__ void run_softmax(SmemCtl<C> &sc, const FwdParams &p, uint32_t tmem, i
           m_ref = mxs;
         }
         const float neg_m = (m_ref == -CUDART_INF_F) ? 0.f : -m_ref;
-        if (full) {
-          // Packed fp32 pairs; one pair in kPolyEvery goes through the FMA-pipe exp2.
+        if (rk) {
+          // Packed fp32 pairs; the pairs kPolyMask selects go through the FMA-pipe exp2. Masked
+          // columns hold -inf and give 0 (MUFU) or 2^-125 (polynomial), i.e. 0 in fp16.
           const uint64_t scp = f2(sc_log2, sc_log2);
           const uint64_t nmp = f2(neg_m, neg_m);
-          uint64_t acc = f2(0.f, 0.f);
-  #pragma unroll
+          uint64_t acc[4] = {f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f)};
+#pragma unroll
           for (int c = 0; c < NCH; ++c) {
-            uint32_t y[32];
-            if (c + 1 < NCH) tmem_ld32(s_addr + (c + 1) * 32, y);
-            reg_fence32(x);
             uint32_t pk[16];
-  #pragma unroll
+#pragma unroll
             for (int e = 0; e < 16; ++e) {
-              const uint64_t xx = fma2(f2(u2f(x[2 * e]), u2f(x[2 * e + 1])), scp, nmp);
+              const int col = c * 32 + 2 * e;
+              const uint64_t xx = fma2(f2(u2f(x[col]), u2f(x[col + 1])), scp, nmp);
               float x0, x1, p0, p1;
               f2_split(xx, x0, x1);
-              if ((e % kPolyEvery) == kPolyEvery - 1) {
+              if ((kPolyMask >> (e % 8)) & 1u) {
                 exp2_poly_x2(x0, x1, p0, p1);
               } else {
                 p0 = ex2_approx(x0);
                 p1 = ex2_approx(x1);
               }
-              acc = add2(acc, f2(p0, p1));
+              acc[e & 3] = add2(acc[e & 3], f2(p0, p1));
               pk[e] = pack_f16x2(p0, p1);
             }
             tmem_st16(s_addr + c * 16, pk);
-            if (c + 1 < NCH) {
-              tmem_wait_ld();
-              reg_fence32(y);
-  #pragma unroll
-              for (int e = 0; e < 32; ++e) x[e] = y[e];
-            }
           }
-          float s0, s1;
-          f2_split(acc, s0, s1);
-          lsum = s0 + s1;
+          float s0, s1, s2, s3, s4, s5, s6, s7;
+          f2_split(acc[0], s0, s1);
+          f2_split(acc[1], s2, s3);
+          f2_split(acc[2], s4, s5);
+          f2_split(acc[3], s6, s7);
+          lsum = ((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7));
         } else {
-  #pragma unroll
-          for (int c = 0; c < NCH; ++c) {
-            uint32_t y[32];
-            if (rk && c + 1 < NCH) tmem_ld32(s_addr + (c + 1) * 32, y);
-            uint32_t pk[16];
-  #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const int col = c * 32 + 2 * e;
-              const float p0 = (rk && col < ncol) ? ex2_approx(fmaf(u2f(x[2 * e]), sc_log2, neg_m)) : 0.f;
-              const float p1 = (rk && col + 1 < ncol) ? ex2_approx(fmaf(u2f(x[2 * e + 1]), sc_log2, neg_m)) : 0.f;
-              lsum += p0 + p1;
-              pk[e] = pack_f16x2(p0, p1);
-            }
-            tmem_st16(s_addr + c * 16, pk);
-            if (rk && c + 1 < NCH) {
-              tmem_wait_ld();
-              reg_fence32(y);
-  #pragma unroll
-              for (int e = 0; e < 32; ++e) x[e] = y[e];
-            }
-          }
+          // This row's query block does not keep the block (two query blocks per tile): P = 0.
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) pk[e] = 0u;
+#pragma unroll
+          for (int c = 0; c < NCH; ++c) tmem_st16(s_addr + c * 16, pk);
         }
       } else if constexpr (TOKEN) {
         softmax_pseudo_tile<BK>(s_addr, j & (kPseudoFlag - 1), rs.kmask[sb], p.N, p.nKB, sc_log2, m_ref, alpha, lsum);
@@ -1221,10 +1212,13 @@ __global__ void __launch_bounds__(256) gauss_theta_kernel(const float *qbar, con
 
 // Work-item schedule for the attention kernel. Each warp routes one item (query tile)
 // exactly as the kernel's router will and records how many key blocks the tile keeps
-// (its cost; nothing else about the keep sets leaves the chip). The last block to finish
-// then orders the items: groups of `group_heads` consecutive heads in head order (the
-// group's K/V stays resident in L2), and within a group the costliest items first, so
-// the short items fill the end of the kernel instead of long ones starting late.
+// (its cost; the keep sets themselves do not leave the chip). In keep_correct with the
+// block correction it also folds every dropped block of each query block into the
+// correction record (p.corr: M, L and C, O(d) per query block), so that the attention
+// kernel's router only takes keep decisions. The last block to finish then orders the
+// items: groups of `group_heads` consecutive heads in head order (the group's K/V stays
+// resident in L2), and within a group the costliest items first, so the short items
+// fill the end of the kernel instead of long ones starting late.
 template <int D, int BQ, int BK, int SUBQ>
 __global__ void __launch_bounds__(256) plan_kernel(const FwdParams p, int *cost, int *order, unsigned int *done,
                                                    int group_heads) {
@@ -1244,9 +1238,20 @@ __global__ void __launch_bounds__(256) plan_kernel(const FwdParams p, int *cost,
     __syncwarp();
     float cacc[D / 32];
     float lacc, M;
+    const bool correct = (p.mode == 2) && !p.token_corr;
     for (int sb = 0; sb < SUBQ; ++sb) {
       const int qb = tile * SUBQ + sb;
-      if (qb < p.nQB) route_block<D, BQ, BK>(p, bh, qb, lane, false, mask[warp][sb], cacc, lacc, M);
+      if (qb >= p.nQB) continue;
+      route_block<D, BQ, BK>(p, bh, qb, lane, correct, mask[warp][sb], cacc, lacc, M);
+      if (correct) {
+        float *rec = p.corr + (static_cast<size_t>(bh) * p.nQB + qb) * corr_stride<D>();
+#pragma unroll
+        for (int e = 0; e < D / 32; ++e) rec[4 + lane * (D / 32) + e] = cacc[e];
+        if (lane == 0) {
+          rec[0] = M;
+          rec[1] = lacc;
+        }
+      }
     }
     __syncwarp();
     int cnt = 0;

@@ -233,6 +233,13 @@ __device__ __forceinline__ void reg_fence32(uint32_t (&r)[32]) {
   for (int i = 0; i < 32; ++i) asm volatile("" : "+r"(r[i]));
 }
 
+// The same for an array of any length.
+template <int W>
+__device__ __forceinline__ void reg_fence(uint32_t (&r)[W]) {
+#pragma unroll
+  for (int i = 0; i < W; ++i) asm volatile("" : "+r"(r[i]));
+}
+
 // Per-warpgroup register budget (every warp of a warpgroup executes the same one).
 // An increase draws on the registers released by decreases in the same block.
 template <int N>

@@ -27,7 +27,7 @@ int nblocks(int N, int blk) { return (N + blk - 1) / blk; }
 bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 struct WsLayout {
-  size_t qbar, kbar, vbar, v16, cost, order, kmom, theta, kbar16, vbar16, total;
+  size_t qbar, kbar, vbar, v16, cost, order, kmom, theta, kbar16, vbar16, corr, total;
 };
 
 int check_shape(int B, int H, int N, int d, int Bq, int Bk) {
@@ -53,7 +53,8 @@ WsLayout ws_layout(int B, int H, int N, int d, int Bq, int Bk) {
   w.theta = w.kmom + align_up(bh * (d + static_cast<size_t>(d) * d) * sizeof(float), kAlign);
   w.kbar16 = w.theta + align_up(bh * nblocks(N, Bq) * sizeof(float), kAlign);  // token-to-block correction
   w.vbar16 = w.kbar16 + align_up(bh * nblocks(N, Bk) * d * 2, kAlign);
-  w.total = w.vbar16 + align_up(bh * nblocks(N, Bk) * d * 2, kAlign);
+  w.corr = w.vbar16 + align_up(bh * nblocks(N, Bk) * d * 2, kAlign);  // block correction per query block
+  w.total = w.corr + align_up(bh * nblocks(N, Bq) * (d + 4) * sizeof(float), kAlign);
   return w;
 }
 
@@ -372,6 +373,7 @@ int forward_impl(const void *q, const void *k, const void *v, void *out, int B, 
   p.n_sink_blocks = nblocks(n_sink, Bk);
   p.token_corr = token ? 1 : 0;
   p.n_pseudo = token ? nblocks(nKB, Bk) : 0;
+  p.corr = reinterpret_cast<float *>(ws + wl.corr);
   if (mode != SOLATTN_DENSE && rule != kRunningMax) {
     float *kmom = reinterpret_cast<float *>(ws + wl.kmom);
     float *theta = reinterpret_cast<float *>(ws + wl.theta);
