@@ -366,6 +366,62 @@ def keep_sets_gaussian(q, k, Bq: int, Bk: int, beta: float, variant: str = "exac
     return keep, margin, sbar
 
 
+# ----------------------------------------------------------------- top-k and top-p routing
+#
+# The routing rules the pages compare Sol-Attn's on-the-fly thresholding against
+# (paperlayer summary "Sol-Attn: Accelerating Video Generation Inference via On-the-Fly
+# Attention Sparsification", §2 Block-Sparse Attention: top-k keeps a fixed budget of the
+# top-ranked blocks, top-p a dynamic one by cumulative probability mass, and both need
+# the whole proxy row; §4 Experiments, "Efficient On-the-Fly Sparsification": routing
+# measured against both). Readings (the pages do not fix them): top-k keeps the k blocks
+# with the largest proxies of each query block's row; top-p keeps the smallest set of
+# heaviest blocks whose share of the row's mass reaches p, where block j's mass is
+# n_j e^{s_ij} (its attention mass under the same zeroth-order approximation as the
+# correction; with equal block sizes this is the softmax of the proxies). Ties go to the
+# lower block index in both.
+
+def rank_desc(s_row: np.ndarray) -> np.ndarray:
+    """Block indices of one proxy row, largest proxy first, lower index first on ties."""
+    return np.lexsort((np.arange(s_row.shape[0]), -s_row))
+
+
+def topk_keep(sbar: np.ndarray, k: int) -> np.ndarray:
+    """Keep the min(k, nKB) largest proxies of every row: [..., nQB, nKB] -> bool."""
+    keep = np.zeros(sbar.shape, dtype=bool)
+    flat_s = sbar.reshape(-1, sbar.shape[-1])
+    flat_k = keep.reshape(-1, sbar.shape[-1])
+    for r in range(flat_s.shape[0]):
+        flat_k[r, rank_desc(flat_s[r])[:k]] = True
+    return keep
+
+
+def topp_keep(sbar: np.ndarray, counts: np.ndarray, p: float) -> np.ndarray:
+    """Rank the blocks of a row by mass n_j e^{s_ij} (largest first) and keep the shortest
+    prefix whose mass reaches p of the row's total: a block is kept iff the mass ranked
+    before it is < p * total."""
+    keep = np.zeros(sbar.shape, dtype=bool)
+    flat_s = sbar.reshape(-1, sbar.shape[-1])
+    flat_k = keep.reshape(-1, sbar.shape[-1])
+    log_n = np.log(counts)
+    for r in range(flat_s.shape[0]):
+        order = rank_desc(flat_s[r] + log_n)  # by mass, largest first
+        w = np.exp(flat_s[r][order] + log_n[order] - (flat_s[r] + log_n).max())
+        before = np.concatenate([[0.0], np.cumsum(w)[:-1]])
+        flat_k[r, order[before < p * w.sum()]] = True
+    return keep
+
+
+def keep_sets_topk(q, k, Bq: int, Bk: int, kb: int):
+    """Top-k keep sets from the block proxies (see above): [B, H, nQB, nKB] bool."""
+    return topk_keep(proxy(pool(as_f64(q), Bq), pool(as_f64(k), Bk)), kb)
+
+
+def keep_sets_topp(q, k, Bq: int, Bk: int, p: float):
+    """Top-p keep sets from the block proxies (see above): [B, H, nQB, nKB] bool."""
+    q, k = as_f64(q), as_f64(k)
+    return topp_keep(proxy(pool(q, Bq), pool(k, Bk)), valid_counts(q.shape[-2], Bk).astype(np.float64), p)
+
+
 def sample_qblocks(B, H, nQB, Bq, Bk, nKB, per_head=64, seed=0):
     """Seeded sample of query blocks per head, plus block 0, the last (ragged) one and
     the blocks whose diagonal is at the extremes."""

@@ -417,8 +417,52 @@ def pin_kept_per_head():
     assert np.array_equal(ref.kept_per_head(dense), np.full((B, H), nQB * nKB))
 
 
+def pin_topk():
+    """Top-k: a hand-worked row with a tie (lower index wins), and on random rows exactly
+    min(k, nKB) blocks kept, none of them below a dropped one."""
+    s = np.array([[3.0, 1.0, 3.0, 2.0]])
+    assert ref.topk_keep(s, 2).tolist() == [[True, False, True, False]]
+    assert ref.topk_keep(s, 1).tolist() == [[True, False, False, False]]
+    assert ref.topk_keep(s, 3).tolist() == [[True, False, True, True]]
+    assert ref.topk_keep(s, 9).all()
+    rng = np.random.default_rng(23)
+    s = rng.standard_normal((3, 7, 29))
+    for k in (1, 5, 29):
+        keep = ref.topk_keep(s, k)
+        assert (keep.sum(-1) == k).all()
+        lo = np.where(keep, s, np.inf).min(-1)
+        hi = np.where(keep, -np.inf, s).max(-1)
+        assert (lo >= hi).all()
+
+
+def pin_topp():
+    """Top-p: a hand-worked row (block sizes 2, 2, 2, 1; proxies ln 4, 0, ln 2, ln 8; masses
+    n_j e^s = 8, 2, 4, 8 of 22; rank 0, 3, 2, 1) and, on random rows, kept mass >= p of the
+    total while the kept set without its lightest block stays below."""
+    s = np.array([[math.log(4.0), 0.0, math.log(2.0), math.log(8.0)]])
+    n = np.array([2.0, 2.0, 2.0, 1.0])
+    assert ref.topp_keep(s, n, 0.5).tolist() == [[True, False, False, True]]     # 0 + 8 < 11 <= 16
+    assert ref.topp_keep(s, n, 0.75).tolist() == [[True, False, True, True]]     # 16 < 16.5
+    assert ref.topp_keep(s, n, 16.0 / 22.0).tolist() == [[True, False, False, True]]  # exactly 16: not below
+    assert ref.topp_keep(s, n, 1.0).all()
+    assert ref.topp_keep(s, n, 1e-9).tolist() == [[True, False, False, False]]   # the heaviest (tie: lower index)
+    rng = np.random.default_rng(29)
+    s = rng.standard_normal((2, 5, 33)) * 2.0
+    n = np.full(33, 64.0)
+    n[-1] = 17.0
+    for p in (0.3, 0.8, 0.95):
+        keep = ref.topp_keep(s, n, p)
+        w = n * np.exp(s)
+        kept = np.where(keep, w, 0.0).sum(-1)
+        assert (kept >= p * w.sum(-1) - 1e-12).all()
+        lightest = np.where(keep, w, np.inf).min(-1)
+        assert (kept - lightest < p * w.sum(-1)).all()
+        hi_drop = np.where(keep, -np.inf, w).max(-1)
+        assert (lightest >= hi_drop).all()
+
+
 PINS += [pin_gaussian_matches_row_statistics, pin_gaussian_diagonal_design, pin_gaussian_keep_fraction,
-         pin_gaussian_limits_and_monotone, pin_sinks, pin_token_correction, pin_kept_per_head]
+         pin_gaussian_limits_and_monotone, pin_sinks, pin_token_correction, pin_kept_per_head, pin_topk, pin_topp]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
@@ -534,6 +578,26 @@ def _mut_kept_one_block_axis(keep):
     return keep.sum(axis=-1)[..., 0].astype(np.int64)
 
 
+def _mut_topk_one_more(sbar, k):
+    return ref.__dict__["_orig_topk"](sbar, k + 1)
+
+
+def _mut_topp_not_strict(sbar, counts, p):
+    keep = np.zeros(sbar.shape, dtype=bool)
+    flat_s, flat_k = sbar.reshape(-1, sbar.shape[-1]), keep.reshape(-1, sbar.shape[-1])
+    log_n = np.log(counts)
+    for r in range(flat_s.shape[0]):
+        order = ref.rank_desc(flat_s[r] + log_n)
+        w = np.exp(flat_s[r][order] + log_n[order] - (flat_s[r] + log_n).max())
+        before = np.concatenate([[0.0], np.cumsum(w)[:-1]])
+        flat_k[r, order[before <= p * w.sum()]] = True
+    return keep
+
+
+def _mut_topp_no_counts(sbar, counts, p):
+    return ref.__dict__["_orig_topp"](sbar, np.ones_like(counts), p)
+
+
 MUTANTS = {
     "pool divides by block size": ("pool", _mut_pool_by_blk),
     "proxy without 1/sqrt(d)": ("proxy", _mut_proxy_unscaled),
@@ -554,6 +618,9 @@ MUTANTS = {
     "token correction without n_j": ("correction_terms_token", _mut_token_no_multiplicity),
     "kept count of the dropped blocks": ("kept_per_head", _mut_kept_counts_dropped),
     "kept count of one query block only": ("kept_per_head", _mut_kept_one_block_axis),
+    "top-k keeps one block too many": ("topk_keep", _mut_topk_one_more),
+    "top-p keeps the block that reaches p exactly": ("topp_keep", _mut_topp_not_strict),
+    "top-p without block sizes": ("topp_keep", _mut_topp_no_counts),
 }
 
 
@@ -561,6 +628,8 @@ MUTANTS = {
 def test_planted_mistakes_are_caught(name, monkeypatch):
     attr, fn = MUTANTS[name]
     monkeypatch.setitem(ref.__dict__, "_orig_attend", ref.attend_block)
+    monkeypatch.setitem(ref.__dict__, "_orig_topk", ref.topk_keep)
+    monkeypatch.setitem(ref.__dict__, "_orig_topp", ref.topp_keep)
     monkeypatch.setattr(ref, attr, fn)
     failed = []
     for pin in PINS:
