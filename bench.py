@@ -51,6 +51,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--all-configs", default="tiny,image,video480,video720,long",
+                    help="configurations swept after the timed region (comma-separated; empty: none)")
     ap.add_argument("--heads", type=int, default=0,
                     help="use only this many heads of the configuration (small profiling captures)")
     return ap.parse_args()
@@ -328,6 +330,152 @@ def reference_arm(args, world, rank):
     print(json.dumps(line), flush=True)
 
 
+def issued_flops(mask_bits, N, Bq, Bk, d):
+    """FLOPs the tensor cores issue: every 128-row query tile runs Q K^T and P V over the
+    union of its query blocks' kept key blocks, full 128 x Bk tiles (ragged rows and columns
+    and rows of a query block that did not keep the entry are computed and masked)."""
+    B, H, nQB, nKB = mask_bits.shape
+    sub = 128 // Bq
+    pad = (-nQB) % sub
+    m = np.concatenate([mask_bits, np.zeros((B, H, pad, nKB), dtype=bool)], axis=2) if pad else mask_bits
+    union = m.reshape(B, H, -1, sub, nKB).any(axis=3)
+    return 4.0 * 128 * Bk * d * float(union.sum())
+
+
+def quantiles(x):
+    x = np.asarray(x, dtype=np.float64)
+    return {q: round(float(np.quantile(x, p)), 5) for q, p in
+            (("min", 0.0), ("p10", 0.1), ("p50", 0.5), ("p90", 0.9), ("max", 1.0))} | {"mean": round(float(x.mean()), 5)}
+
+
+def config_sweep(name, dev, stream, peak_tf, reps=5):
+    """One configuration: every (mode, tau) of its sweep timed as whole solattn_forward calls
+    (median of `reps` after 2 warm-up calls), with keep ratios (block and token-weighted),
+    executed, issued and dense-equivalent TFLOP/s, the correction ablation against the dense
+    output at identical keep sets (rel-l2 and cosine similarity of keep_drop and keep_correct,
+    paperlayer summary §4 "Ablations"), the keep-ratio distribution per head and per query
+    block, and torch's bf16 SDPA on the same inputs for context."""
+    import torch
+    from block_sparse_online_b200 import solattn, synth
+    cfg = synth.CONFIGS[name]
+    B, H, N, d = cfg.shape()
+    q, k, v = synth.make_inputs(cfg)
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    del q, k, v
+    ws = solattn.alloc_workspace(B, H, N, d, cfg.Bq, cfg.Bk, dev)
+    out = torch.empty_like(qd)
+    kept = torch.empty((B, H), dtype=torch.int64, device=dev)
+    dense_flops = cfg.dense_flops()
+    bq, bk = block_sizes(N, cfg.Bq), block_sizes(N, cfg.Bk)
+
+    def timed(fn):
+        for _ in range(2):
+            fn()
+        ts = []
+        for _ in range(reps):
+            a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a0.record(stream)
+            fn()
+            a1.record(stream)
+            torch.cuda.synchronize()
+            ts.append(a0.elapsed_time(a1))
+        return statistics.median(ts)
+
+    dense_out, _, _ = solattn.solattn_forward(qd, kd, vd, cfg.Bq, cfg.Bk, 0.0, "dense", workspace=ws)
+    dense_out = dense_out.float()
+    rows = []
+    for mode in ("dense", "keep_drop", "keep_correct"):
+        for tau in ((0.0,) if mode == "dense" else cfg.taus):
+            o, _, m = solattn.solattn_forward(qd, kd, vd, cfg.Bq, cfg.Bk, tau, mode, keep_mask=True, workspace=ws)
+            if solattn.solattn_get_status(ws) != 0:
+                raise RuntimeError(f"{name} {mode} {tau}: device status")
+            bits = unpack(m, cfg.nKB)
+            ms = timed(lambda: solattn.solattn_forward(qd, kd, vd, cfg.Bq, cfg.Bk, tau, mode, out=out,
+                                                       kept_per_head=kept, workspace=ws))
+            ef = executed_flops(bits, N, cfg.Bq, cfg.Bk, d)
+            row = {"mode": mode, "tau": None if (mode == "dense" or math.isinf(tau)) else tau, "ms": round(ms, 4),
+                   "keep_ratio": round(float(bits.mean()), 5),
+                   "keep_ratio_tokens": round(float(np.einsum("bhij,i,j->", bits.astype(np.float64), bq, bk)
+                                                    / (B * H * N * N)), 5),
+                   "exec_tflops": round(ef / (ms * 1e-3) / 1e12, 2),
+                   "exec_frac_of_peak": round(ef / (ms * 1e-3) / 1e12 / peak_tf, 4),
+                   "dense_equiv_tflops": round(dense_flops / (ms * 1e-3) / 1e12, 2)}
+            if cfg.Bq == 64:
+                isf = issued_flops(bits, N, cfg.Bq, cfg.Bk, d)
+                row["issued_tflops"] = round(isf / (ms * 1e-3) / 1e12, 2)
+                row["issued_over_executed"] = round(isf / ef, 4)
+            if mode != "dense":
+                x, y = o.float().flatten(), dense_out.flatten()
+                row["rel_l2_vs_dense"] = round(float(torch.linalg.vector_norm(x - y) / torch.linalg.vector_norm(y)), 6)
+                row["cos_sim_vs_dense"] = round(float(torch.nn.functional.cosine_similarity(x, y, dim=0)), 6)
+                if mode == "keep_correct":
+                    per_head = bits.mean(axis=(-1, -2)).reshape(-1)
+                    per_qb = bits.mean(axis=-1).reshape(-1)
+                    row["keep_ratio_per_head"] = quantiles(per_head)
+                    row["keep_ratio_per_query_block"] = quantiles(per_qb)
+                    row["keep_ratio_per_query_block_hist"] = np.histogram(per_qb, bins=10, range=(0.0, 1.0))[0].tolist()
+            rows.append(row)
+    # Context: torch's fused bf16 attention on the same inputs. The unfused math backend would
+    # materialise N x N scores (hundreds of GB at the long shape), so it is excluded.
+    from torch.nn.attention import SDPBackend, sdpa_kernel
+    try:
+        with sdpa_kernel([SDPBackend.CUDNN_ATTENTION, SDPBackend.FLASH_ATTENTION, SDPBackend.EFFICIENT_ATTENTION]):
+            sdpa_ms = timed(lambda: torch.nn.functional.scaled_dot_product_attention(qd, kd, vd))
+        sdpa = {"ms": round(sdpa_ms, 4), "tflops": round(dense_flops / (sdpa_ms * 1e-3) / 1e12, 2),
+                "note": "torch.nn.functional.scaled_dot_product_attention, bf16, same inputs (library kernel; "
+                        "context only)"}
+    except RuntimeError as e:
+        sdpa = {"unavailable": str(e).splitlines()[0][:200]}
+    res = {"workload": cfg.note, "shape": [B, H, N, d], "Bq": cfg.Bq, "Bk": cfg.Bk, "rows": rows,
+           "torch_sdpa_bf16": sdpa}
+    del qd, kd, vd, ws, out, dense_out
+    torch.cuda.empty_cache()
+    return res
+
+
+def routing_overhead(cfg, qd, kd, tau, stream):
+    """The routing stage alone on the pooled blocks of the timed inputs (paperlayer summary
+    §4, "Efficient On-the-Fly Sparsification"): the running-max rule with the proxies kept on
+    chip, against top-k and top-p routers that first write the proxy map to HBM. k is the
+    mean number of blocks our rule keeps per query block at this tau; top-p is timed at two
+    masses. CUDA events, median of 10 after 3 warm-up calls each."""
+    import torch
+    from block_sparse_online_b200 import solattn
+    N = cfg.N
+    qb, kb = solattn.solattn_pool(qd, cfg.Bq), solattn.solattn_pool(kd, cfg.Bk)
+    mask = solattn.solattn_route_keep(qb, kb, N, cfg.Bq, cfg.Bk, tau)
+    bits = unpack(mask, cfg.nKB)
+    kk = max(1, int(round(float(bits.sum(-1).mean()))))
+    smap = torch.empty(solattn.solattn_proxy_map_bytes(cfg.B, cfg.H, N, cfg.Bq, cfg.Bk) // 4, dtype=torch.float32,
+                       device=qd.device)
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        ts = []
+        for _ in range(10):
+            a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a0.record(stream)
+            fn()
+            a1.record(stream)
+            torch.cuda.synchronize()
+            ts.append(a0.elapsed_time(a1))
+        return statistics.median(ts)
+
+    ours = timed(lambda: solattn.solattn_route_keep(qb, kb, N, cfg.Bq, cfg.Bk, tau, keep_mask=mask))
+    topk = timed(lambda: solattn.solattn_route_topk(qb, kb, N, cfg.Bq, cfg.Bk, kk, keep_mask=mask, proxy_map=smap))
+    out = {"tau": tau, "keep_ratio": round(float(bits.mean()), 5), "ours_ms": round(ours, 4),
+           "topk": {"k": kk, "ms": round(topk, 4), "slowdown_vs_ours": round(topk / ours, 2)}, "topp": [],
+           "proxy_map_bytes": int(smap.numel() * 4),
+           "pages": "routing 11.5x faster than top-k and 32.7x faster than top-p (paperlayer summary, section 4)"}
+    for pm in (0.9, 0.99):
+        t = timed(lambda: solattn.solattn_route_topp(qb, kb, N, cfg.Bq, cfg.Bk, pm, keep_mask=mask, proxy_map=smap))
+        kr = float(unpack(mask, cfg.nKB).mean())
+        out["topp"].append({"p": pm, "ms": round(t, 4), "keep_ratio": round(kr, 5),
+                            "slowdown_vs_ours": round(t / ours, 2)})
+    return out
+
+
 def e2e_measure(args, cfg, q, k, v, dev, stream, world, barrier, dense_flops, elem):
     """Same metric through the host entry point: pinned host q/k/v in, host output out,
     host<->device copies inside the timed region."""
@@ -441,6 +589,8 @@ def main():
         e2e = e2e_measure(args, cfg, q, k, v, dev, stream, world, barrier, dense_flops, elem)
 
     sweep = []
+    routing = None
+    configs = {}
     if not args.no_sweep and rank == 0:
         for mode in ("keep_drop", "keep_correct"):
             for tau in cfg.taus:
@@ -518,6 +668,10 @@ def main():
         sweep.append({"mode": "dense", "tau": None, "ms": round(ms, 4), "keep_ratio": 1.0,
                       "exec_tflops": round(dense_flops / (ms * 1e-3) / 1e12, 2),
                       "dense_equiv_tflops": round(dense_flops / (ms * 1e-3) / 1e12, 2)})
+        routing = routing_overhead(cfg, qd, kd, args.tau, stream)
+        peak_tf0, _, _ = measured_peaks()
+        for name in (args.all_configs.split(",") if args.all_configs else []):
+            configs[name] = config_sweep(name, dev, stream, peak_tf0)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -547,6 +701,8 @@ def main():
             "clocks": clk,
             "cpu_baseline": cpu,
             "sweep": sweep,
+            "routing_overhead": routing,
+            "configs": configs,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -10,6 +10,7 @@
 
 #include "attn_kernel.cuh"
 #include "pool_kernel.cuh"
+#include "route_kernels.cuh"
 #include "solattn.h"
 
 namespace {
@@ -403,6 +404,59 @@ int forward_impl(const void *q, const void *k, const void *v, void *out, int B, 
   return SOLATTN_OK;
 }
 
+// ---- routing on its own (routing-overhead measurement)
+
+template <int D, int BQ, int BK>
+int launch_route_t(const FwdParams &p, uint32_t *mask, int n_rows, cudaStream_t st) {
+  route_kernel<D, BQ, BK><<<(n_rows + 7) / 8, 256, 0, st>>>(p, mask, n_rows);
+  return cudaGetLastError() == cudaSuccess ? SOLATTN_OK : SOLATTN_ECUDA;
+}
+
+int launch_route(int d, int Bq, int Bk, const FwdParams &p, uint32_t *mask, int n_rows, cudaStream_t st) {
+  if (d == 128) {
+    if (Bq == 128) return Bk == 128 ? launch_route_t<128, 128, 128>(p, mask, n_rows, st)
+                                    : launch_route_t<128, 128, 64>(p, mask, n_rows, st);
+    return Bk == 128 ? launch_route_t<128, 64, 128>(p, mask, n_rows, st) : launch_route_t<128, 64, 64>(p, mask, n_rows, st);
+  }
+  if (Bq == 128) return Bk == 128 ? launch_route_t<64, 128, 128>(p, mask, n_rows, st)
+                                  : launch_route_t<64, 128, 64>(p, mask, n_rows, st);
+  return Bk == 128 ? launch_route_t<64, 64, 128>(p, mask, n_rows, st) : launch_route_t<64, 64, 64>(p, mask, n_rows, st);
+}
+
+template <int P>
+int launch_select_t(const float *smap, uint32_t *mask, int rows, int nKB, int N, int Bk, int topp, int k, float pm,
+                    cudaStream_t st) {
+  select_kernel<P><<<rows, 512, 0, st>>>(smap, mask, nKB, N, Bk, topp, k, pm);
+  return cudaGetLastError() == cudaSuccess ? SOLATTN_OK : SOLATTN_ECUDA;
+}
+
+// Materialise the proxy map, then select per row (top-k: topp = 0, k; top-p: topp = 1, pm).
+int route_select(const float *qbar, const float *kbar, int B, int H, int N, int d, int Bq, int Bk, int topp, int k,
+                 float pm, float *proxy_map, size_t map_bytes, uint32_t *keep_mask, void *stream) {
+  if (!qbar || !kbar || !proxy_map || !keep_mask) return SOLATTN_EINVAL;
+  const int rc = check_shape(B, H, N, d, Bq, Bk);
+  if (rc != SOLATTN_OK) return rc;
+  if (!aligned(qbar, 16) || !aligned(kbar, 16) || !aligned(proxy_map, 4) || !aligned(keep_mask, 4)) return SOLATTN_EINVAL;
+  const int BH = B * H, nQB = nblocks(N, Bq), nKB = nblocks(N, Bk);
+  if (map_bytes < static_cast<size_t>(BH) * nQB * nKB * sizeof(float)) return SOLATTN_EWORKSPACE;
+  DeviceInfo di;
+  if (device_info(&di) != SOLATTN_OK) return SOLATTN_ECUDA;
+  if (di.major != 10) return SOLATTN_EUNSUPPORTED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const dim3 grid((nKB + 63) / 64, (nQB + 63) / 64, BH);
+  if (d == 128)
+    proxy_map_kernel<128><<<grid, 256, 0, st>>>(qbar, kbar, proxy_map, nQB, nKB);
+  else
+    proxy_map_kernel<64><<<grid, 256, 0, st>>>(qbar, kbar, proxy_map, nQB, nKB);
+  if (cudaGetLastError() != cudaSuccess) return SOLATTN_ECUDA;
+  const int rows = BH * nQB;
+  if (nKB <= 64) return launch_select_t<64>(proxy_map, keep_mask, rows, nKB, N, Bk, topp, k, pm, st);
+  if (nKB <= 128) return launch_select_t<128>(proxy_map, keep_mask, rows, nKB, N, Bk, topp, k, pm, st);
+  if (nKB <= 256) return launch_select_t<256>(proxy_map, keep_mask, rows, nKB, N, Bk, topp, k, pm, st);
+  if (nKB <= 512) return launch_select_t<512>(proxy_map, keep_mask, rows, nKB, N, Bk, topp, k, pm, st);
+  return launch_select_t<1024>(proxy_map, keep_mask, rows, nKB, N, Bk, topp, k, pm, st);
+}
+
 }  // namespace
 
 extern "C" {
@@ -548,6 +602,45 @@ int solattn_selftest_exp2(const float *x, float *y, int n, void *stream) {
   const int pairs = (n + 1) / 2;
   exp2_selftest_kernel<<<(pairs + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n);
   return cudaGetLastError() == cudaSuccess ? SOLATTN_OK : SOLATTN_ECUDA;
+}
+
+int solattn_route_keep(const float *qbar, const float *kbar, int B, int H, int N, int d, int Bq, int Bk, float tau,
+                       uint32_t *keep_mask, void *stream) {
+  if (!qbar || !kbar || !keep_mask) return SOLATTN_EINVAL;
+  const int rc = check_shape(B, H, N, d, Bq, Bk);
+  if (rc != SOLATTN_OK) return rc;
+  if (!(tau >= 0.f)) return SOLATTN_EINVAL;
+  if (!aligned(qbar, 16) || !aligned(kbar, 16) || !aligned(keep_mask, 4)) return SOLATTN_EINVAL;
+  DeviceInfo di;
+  if (device_info(&di) != SOLATTN_OK) return SOLATTN_ECUDA;
+  if (di.major != 10) return SOLATTN_EUNSUPPORTED;
+  FwdParams p{};
+  p.N = N;
+  p.nQB = nblocks(N, Bq);
+  p.nKB = nblocks(N, Bk);
+  p.mode = SOLATTN_KEEP_DROP;  // keep decisions only
+  p.tau = tau;
+  p.qbar = qbar;
+  p.kbar = kbar;
+  const int rows = B * H * p.nQB;
+  return launch_route(d, Bq, Bk, p, keep_mask, rows, static_cast<cudaStream_t>(stream));
+}
+
+size_t solattn_proxy_map_bytes(int B, int H, int N, int Bq, int Bk) {
+  if (check_shape(B, H, N, 128, Bq, Bk) != SOLATTN_OK) return 0;
+  return static_cast<size_t>(B) * H * nblocks(N, Bq) * nblocks(N, Bk) * sizeof(float);
+}
+
+int solattn_route_topk(const float *qbar, const float *kbar, int B, int H, int N, int d, int Bq, int Bk, int k,
+                       float *proxy_map, size_t map_bytes, uint32_t *keep_mask, void *stream) {
+  if (k < 1) return SOLATTN_EINVAL;
+  return route_select(qbar, kbar, B, H, N, d, Bq, Bk, 0, k, 0.f, proxy_map, map_bytes, keep_mask, stream);
+}
+
+int solattn_route_topp(const float *qbar, const float *kbar, int B, int H, int N, int d, int Bq, int Bk, float p,
+                       float *proxy_map, size_t map_bytes, uint32_t *keep_mask, void *stream) {
+  if (!(p > 0.f && p <= 1.f)) return SOLATTN_EINVAL;
+  return route_select(qbar, kbar, B, H, N, d, Bq, Bk, 1, 0, p, proxy_map, map_bytes, keep_mask, stream);
 }
 
 const char *solattn_strerror(int status) {

@@ -30,6 +30,7 @@ EXPORTS = ("solattn_workspace_size", "solattn_pool", "solattn_forward", "solattn
            "solattn_get_status",
            "solattn_host_workspace_size", "solattn_forward_host", "solattn_watchdog_selftest",
            "solattn_selftest_exp2", "solattn_forward_noalloc", "solattn_forward_gaussian", "solattn_forward_ex",
+           "solattn_route_keep", "solattn_proxy_map_bytes", "solattn_route_topk", "solattn_route_topp",
            "solattn_strerror")
 GAUSS_VARIANTS = {"exact": 0, "diag": 1}  # solattn_gauss_variant
 RULES = {"running_max": 0, "gauss_exact": 1, "gauss_diag": 2}  # solattn_rule
@@ -83,6 +84,14 @@ def _load():
     lib.solattn_forward_noalloc.restype = i
     lib.solattn_selftest_exp2.argtypes = [vp, vp, i, vp]
     lib.solattn_selftest_exp2.restype = i
+    lib.solattn_route_keep.argtypes = [vp, vp, i, i, i, i, i, i, f, vp, vp]
+    lib.solattn_route_keep.restype = i
+    lib.solattn_proxy_map_bytes.argtypes = [i, i, i, i, i]
+    lib.solattn_proxy_map_bytes.restype = sz
+    lib.solattn_route_topk.argtypes = [vp, vp, i, i, i, i, i, i, i, vp, sz, vp, vp]
+    lib.solattn_route_topk.restype = i
+    lib.solattn_route_topp.argtypes = [vp, vp, i, i, i, i, i, i, f, vp, sz, vp, vp]
+    lib.solattn_route_topp.restype = i
     lib.solattn_strerror.argtypes = [i]
     lib.solattn_strerror.restype = ctypes.c_char_p
     return lib
@@ -354,6 +363,74 @@ def solattn_forward_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, B
                                           _stream(stream, q.device))
     _check(rc, "solattn_forward_noalloc")
     return out, kept_per_head
+
+
+def _route_args(qbar: torch.Tensor, kbar: torch.Tensor, N: int, Bq: int, Bk: int, keep_mask):
+    if qbar.dim() != 4 or kbar.dim() != 4:
+        raise ValueError("qbar and kbar must be [B, H, nB, d]")
+    B, H, nQB, d = (int(x) for x in qbar.shape)
+    nKB = -(-N // Bk)
+    if nQB != -(-N // Bq) or tuple(kbar.shape) != (B, H, nKB, d):
+        raise ValueError("qbar / kbar do not match N, Bq, Bk")
+    for name, t in (("qbar", qbar), ("kbar", kbar)):
+        _check_buffer(t, name, (torch.float32,), t.numel(), qbar.device)
+    if keep_mask is None:
+        keep_mask = torch.empty((B, H, nQB, -(-nKB // 32)), dtype=torch.int32, device=qbar.device)
+    _check_buffer(keep_mask, "keep_mask", (torch.int32, torch.uint32), B * H * nQB * (-(-nKB // 32)), qbar.device)
+    return B, H, d, keep_mask
+
+
+def solattn_route_keep(qbar: torch.Tensor, kbar: torch.Tensor, N: int, Bq: int, Bk: int, tau: float,
+                       keep_mask: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """The running-maximum routing rule alone on pooled blocks (fp32 [B, H, nB, d]); returns the
+    keep bits [B, H, nQB, ceil(nKB/32)] (int32 storage of u32 words)."""
+    B, H, d, keep_mask = _route_args(qbar, kbar, N, Bq, Bk, keep_mask)
+    with torch.cuda.device(qbar.device):
+        rc = _lib.solattn_route_keep(qbar.data_ptr(), kbar.data_ptr(), B, H, N, d, Bq, Bk, ctypes.c_float(float(tau)),
+                                     keep_mask.data_ptr(), _stream(stream, qbar.device))
+    _check(rc, "solattn_route_keep")
+    return keep_mask
+
+
+def solattn_proxy_map_bytes(B, H, N, Bq, Bk) -> int:
+    """Bytes of the fp32 proxy map the top-k and top-p routers write (0 if the shape is invalid)."""
+    return int(_lib.solattn_proxy_map_bytes(B, H, N, Bq, Bk))
+
+
+def _proxy_map(B, H, N, Bq, Bk, proxy_map, device):
+    n = solattn_proxy_map_bytes(B, H, N, Bq, Bk)
+    if proxy_map is None:
+        proxy_map = torch.empty(n // 4, dtype=torch.float32, device=device)
+    _check_buffer(proxy_map, "proxy_map", (torch.float32,), n // 4, device)
+    return proxy_map
+
+
+def solattn_route_topk(qbar: torch.Tensor, kbar: torch.Tensor, N: int, Bq: int, Bk: int, k: int,
+                       keep_mask: torch.Tensor | None = None, proxy_map: torch.Tensor | None = None, stream=None):
+    """Top-k routing (materialised proxy map, the k largest proxies per query block).
+    Returns (keep bits, proxy map)."""
+    B, H, d, keep_mask = _route_args(qbar, kbar, N, Bq, Bk, keep_mask)
+    proxy_map = _proxy_map(B, H, N, Bq, Bk, proxy_map, qbar.device)
+    with torch.cuda.device(qbar.device):
+        rc = _lib.solattn_route_topk(qbar.data_ptr(), kbar.data_ptr(), B, H, N, d, Bq, Bk, int(k),
+                                     proxy_map.data_ptr(), proxy_map.numel() * 4, keep_mask.data_ptr(),
+                                     _stream(stream, qbar.device))
+    _check(rc, "solattn_route_topk")
+    return keep_mask, proxy_map
+
+
+def solattn_route_topp(qbar: torch.Tensor, kbar: torch.Tensor, N: int, Bq: int, Bk: int, p: float,
+                       keep_mask: torch.Tensor | None = None, proxy_map: torch.Tensor | None = None, stream=None):
+    """Top-p routing (materialised proxy map; the heaviest blocks until their share of the
+    row's mass reaches p). Returns (keep bits, proxy map)."""
+    B, H, d, keep_mask = _route_args(qbar, kbar, N, Bq, Bk, keep_mask)
+    proxy_map = _proxy_map(B, H, N, Bq, Bk, proxy_map, qbar.device)
+    with torch.cuda.device(qbar.device):
+        rc = _lib.solattn_route_topp(qbar.data_ptr(), kbar.data_ptr(), B, H, N, d, Bq, Bk, ctypes.c_float(float(p)),
+                                     proxy_map.data_ptr(), proxy_map.numel() * 4, keep_mask.data_ptr(),
+                                     _stream(stream, qbar.device))
+    _check(rc, "solattn_route_topp")
+    return keep_mask, proxy_map
 
 
 def solattn_selftest_exp2(x: torch.Tensor, stream=None) -> torch.Tensor:

@@ -263,6 +263,41 @@ int solattn_forward_ex(const void *q, const void *k, const void *v, void *out,
                        void *stream);
 
 /*
+ * The routing stage on its own, for the routing-overhead measurement ("Sol-Attn:
+ * Accelerating Video Generation Inference via On-the-Fly Attention Sparsification",
+ * paperlayer summary §4 Experiments, "Efficient On-the-Fly Sparsification": routing that
+ * consumes proxy scores on chip, against top-k and top-p routing, which materialise the
+ * proxy map and traverse its rows; §2 Block-Sparse Attention). The three routers read the
+ * same pooled blocks and write keep bits in the layout of solattn_stats.keep_mask:
+ *
+ *   qbar, kbar  device fp32 [B][H][nQB][d] and [B][H][nKB][d] (block means, as written by
+ *               solattn_pool with blk = Bq and Bk), 16-byte aligned
+ *   keep_mask   device u32 [B][H][nQB][ceil(nKB/32)], written
+ *   proxy_map   device fp32 scratch of solattn_proxy_map_bytes(...) bytes (map_bytes), which
+ *               the top-k and top-p routers fill with s_ij = q_i . k_j / sqrt(d)
+ *
+ * solattn_route_keep: the running-maximum rule of solattn_forward (same visit order, same
+ *   tau), computed as the forward kernel's router does, with no proxy leaving the chip.
+ * solattn_route_topk: keeps the min(k, nKB) key blocks with the largest proxies of every
+ *   query block (ties: lower block index). k >= 1.
+ * solattn_route_topp: ranks the key blocks of a query block by mass n_j e^{s_ij} (n_j valid
+ *   keys of block j; ties: lower index) and keeps the shortest prefix whose share of the
+ *   row's total mass reaches p (a block is kept iff the mass ranked before it is below
+ *   p times the total). 0 < p <= 1.
+ * The readings of top-k and top-p are this library's (the pages name the rules only).
+ * Errors: null or misaligned pointers, tau < 0 or NaN, k < 1, p outside (0, 1] ->
+ * SOLATTN_EINVAL; a short proxy_map -> SOLATTN_EWORKSPACE; otherwise as solattn_forward.
+ * Asynchronous on `stream`.
+ */
+int solattn_route_keep(const float *qbar, const float *kbar, int B, int H, int N, int d, int Bq, int Bk,
+                       float tau, uint32_t *keep_mask, void *stream);
+size_t solattn_proxy_map_bytes(int B, int H, int N, int Bq, int Bk);
+int solattn_route_topk(const float *qbar, const float *kbar, int B, int H, int N, int d, int Bq, int Bk,
+                       int k, float *proxy_map, size_t map_bytes, uint32_t *keep_mask, void *stream);
+int solattn_route_topp(const float *qbar, const float *kbar, int B, int H, int N, int d, int Bq, int Bk,
+                       float p, float *proxy_map, size_t map_bytes, uint32_t *keep_mask, void *stream);
+
+/*
  * Synchronise `stream` and read the device status word of `workspace`
  * (SOLATTN_OK, or SOLATTN_ETIMEOUT if a bounded device-side wait gave up).
  */

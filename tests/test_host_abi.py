@@ -175,3 +175,21 @@ def test_binding_rejects_cpu_tensors():
     q = torch.zeros(1, 1, 64, 64, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         solattn.solattn_forward(q, q, q, 64, 64, 1.0, "keep_drop")
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="placeholder pointers are used only without a GPU")
+def test_routing_entry_points_reject_bad_arguments():
+    L = solattn._lib
+    f = ctypes.c_float
+    args = (4096, 4096, 1, 2, 1000, 64, 64, 64)
+    assert L.solattn_route_keep(None, 4096, *args[2:], f(1.0), 4096, None) == solattn.SOLATTN_EINVAL
+    assert L.solattn_route_keep(*args, f(-1.0), 4096, None) == solattn.SOLATTN_EINVAL
+    assert L.solattn_route_keep(*args, f(float("nan")), 4096, None) == solattn.SOLATTN_EINVAL
+    assert L.solattn_route_keep(4096, 4096, 1, 2, 1000, 96, 64, 64, f(1.0), 4096, None) == solattn.SOLATTN_EUNSUPPORTED
+    need = solattn._lib.solattn_proxy_map_bytes(1, 2, 1000, 64, 64)
+    assert need == 2 * 16 * 16 * 4
+    assert L.solattn_route_topk(*args, 0, 4096, need, 4096, None) == solattn.SOLATTN_EINVAL
+    assert L.solattn_route_topk(*args, 3, 4096, need - 4, 4096, None) == solattn.SOLATTN_EWORKSPACE
+    for p in (0.0, -0.5, 1.5, float("nan")):
+        assert L.solattn_route_topp(*args, f(p), 4096, need, 4096, None) == solattn.SOLATTN_EINVAL
+    assert L.solattn_route_topp(*args, f(0.9), None, need, 4096, None) == solattn.SOLATTN_EINVAL
