@@ -537,6 +537,10 @@ __device__ void run_producer(SmemCtl<C> &sc, const FwdParams &p, uint8_t *q_smem
   const volatile int *ab = &sc.abort_flag;
   uint32_t kv_it = 0, q_it = 0;
   bool ok = true;
+  // L2 priorities: a Q tile is read by one item only; a K or V tile by every query tile of
+  // its head that keeps the block, so it should still be in L2 when the next one needs it.
+  const uint64_t pol_stream = l2_policy_evict_first();
+  const uint64_t pol_reuse = l2_policy_evict_last();
   // Loads one K or V tile of key block j into the next ring slot.
   auto load = [&](int j, bool is_v, int bh) {
     const int slot = kv_it % C::NSLOT;
@@ -553,7 +557,8 @@ __device__ void run_producer(SmemCtl<C> &sc, const FwdParams &p, uint8_t *q_smem
     const int row = (j & (kPseudoFlag - 1)) * C::BK;
 #pragma unroll
     for (int pn = 0; pn < C::PANELS; ++pn)
-      tma_load_3d(smem_u32(dst + pn * (C::BK * 128)), map, smem_u32(&sc.full[slot]), pn * 64, row, bh);
+      tma_load_3d_hint(smem_u32(dst + pn * (C::BK * 128)), map, smem_u32(&sc.full[slot]), pn * 64, row, bh,
+                       pol_reuse);
     ++kv_it;
   };
   for (uint32_t r_it = 0;; ++r_it) {
@@ -569,8 +574,8 @@ __device__ void run_producer(SmemCtl<C> &sc, const FwdParams &p, uint8_t *q_smem
     mbar_arrive_expect_tx(&sc.q_full[qb], C::Q_TILE_BYTES);
 #pragma unroll
     for (int pn = 0; pn < C::PANELS; ++pn)
-      tma_load_3d(smem_u32(q_smem + qb * C::Q_TILE_BYTES + pn * (C::TILE_M * 128)), tm_q, smem_u32(&sc.q_full[qb]),
-                  pn * 64, row0, bh);
+      tma_load_3d_hint(smem_u32(q_smem + qb * C::Q_TILE_BYTES + pn * (C::TILE_M * 128)), tm_q,
+                       smem_u32(&sc.q_full[qb]), pn * 64, row0, bh, pol_stream);
     ++q_it;
     // Ring order = consumption order of the MMA warp: K_0, K_1, then V_u, K_{u+2}.
     const int n = rs.n_union;
@@ -821,6 +826,7 @@ __device__ void run_softmax(SmemCtl<C> &sc, const FwdParams &p, uint32_t tmem, i
   const uint32_t row_bit = 1u << sb;
   uint32_t s_ph = 0;
   uint32_t kv_base = 0;  // ring entries of earlier items (2 per kept block)
+  const uint64_t pol_out = l2_policy_evict_first();
   // One thread per warpgroup returns the ring slots (and the Q buffer) the tensor core
   // has finished reading: the MMA issuers commit only the barrier this warpgroup waits on.
   const bool leader = (threadIdx.x & 127) == 0;
@@ -1000,8 +1006,9 @@ __device__ void run_softmax(SmemCtl<C> &sc, const FwdParams &p, uint32_t tmem, i
           }
           pk[e] = pack_bf16x2(y0 * inv, y1 * inv);
         }
-        dst[(col0 >> 3)] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-        dst[(col0 >> 3) + 1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        // output rows are not read again by this kernel: they should not displace K and V in L2
+        st_global_v4_hint(dst + (col0 >> 3), pk[0], pk[1], pk[2], pk[3], pol_out);
+        st_global_v4_hint(dst + (col0 >> 3) + 1, pk[4], pk[5], pk[6], pk[7], pol_out);
       }
     }
     tc_fence_before_sync();
