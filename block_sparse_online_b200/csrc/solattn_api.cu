@@ -457,6 +457,39 @@ int route_select(const float *qbar, const float *kbar, int B, int H, int N, int 
   return launch_select_t<1024>(proxy_map, keep_mask, rows, nKB, N, Bk, topp, k, pm, st);
 }
 
+// ---- streams and events of solattn_forward_host, created once per device
+
+constexpr int kHostChunks = 16;  // most chunks of heads one host call pipelines
+
+struct HostPipe {
+  std::mutex mu;
+  bool ready = false;
+  cudaStream_t up = nullptr, down = nullptr;
+  cudaEvent_t ev_start = nullptr, ev_end = nullptr;
+  cudaEvent_t ev_up[kHostChunks] = {}, ev_done[kHostChunks] = {};
+};
+HostPipe g_pipe[64];
+
+int host_pipe(HostPipe **out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return SOLATTN_ECUDA;
+  HostPipe &hp = g_pipe[dev];
+  std::lock_guard<std::mutex> lk(hp.mu);
+  if (!hp.ready) {
+    // Each handle is created once; after a failure the next call creates only the rest.
+    auto stream = [](cudaStream_t *x) {
+      return *x || cudaStreamCreateWithFlags(x, cudaStreamNonBlocking) == cudaSuccess;
+    };
+    auto event = [](cudaEvent_t *x) { return *x || cudaEventCreateWithFlags(x, cudaEventDisableTiming) == cudaSuccess; };
+    bool ok = stream(&hp.up) && stream(&hp.down) && event(&hp.ev_start) && event(&hp.ev_end);
+    for (int c = 0; ok && c < kHostChunks; ++c) ok = event(&hp.ev_up[c]) && event(&hp.ev_done[c]);
+    if (!ok) return SOLATTN_ECUDA;
+    hp.ready = true;
+  }
+  *out = &hp;
+  return SOLATTN_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -548,7 +581,8 @@ size_t solattn_host_workspace_size(int B, int H, int N, int d, int Bq, int Bk) {
   const size_t elems = static_cast<size_t>(B) * H * N * d;
   const size_t t = align_up(elems * 2, kAlign);
   const size_t kp = align_up(sizeof(int64_t) * B * H, kAlign);
-  return 4 * t + kp + ws_layout(B, H, N, d, Bq, Bk).total;
+  const size_t sp = align_up(sizeof(int) * kHostChunks, kAlign);
+  return 4 * t + kp + sp + ws_layout(B, H, N, d, Bq, Bk).total;
 }
 
 int solattn_forward_host(const void *q, const void *k, const void *v, void *out, int B, int H, int N, int d,
@@ -557,28 +591,75 @@ int solattn_forward_host(const void *q, const void *k, const void *v, void *out,
   if (!q || !k || !v || !out) return SOLATTN_EINVAL;
   const int rc = check_shape(B, H, N, d, Bq, Bk);
   if (rc != SOLATTN_OK) return rc;
+  if (mode < SOLATTN_DENSE || mode > SOLATTN_KEEP_CORRECT || !(tau >= 0.f)) return SOLATTN_EINVAL;
   const size_t need = solattn_host_workspace_size(B, H, N, d, Bq, Bk);
   if (!dev_scratch || !aligned(dev_scratch, kAlign) || scratch_bytes < need) return SOLATTN_EWORKSPACE;
+  HostPipe *hp = nullptr;
+  const int rp = host_pipe(&hp);
+  if (rp != SOLATTN_OK) return rp;
+  std::lock_guard<std::mutex> lk(hp->mu);  // the pipe's streams and events serve one call at a time
+
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const size_t bytes = static_cast<size_t>(B) * H * N * d * 2;
-  const size_t t = align_up(bytes, kAlign);
+  const int BH = B * H;
+  const size_t head = static_cast<size_t>(N) * d * 2;  // bytes of one head of q, k, v or out
+  const size_t t = align_up(head * BH, kAlign);
   uint8_t *base = static_cast<uint8_t *>(dev_scratch);
   uint8_t *dq = base, *dk = base + t, *dv = base + 2 * t, *dout = base + 3 * t;
   int64_t *dkept = reinterpret_cast<int64_t *>(base + 4 * t);
-  uint8_t *ws = base + 4 * t + align_up(sizeof(int64_t) * B * H, kAlign);
+  int *dstatus = reinterpret_cast<int *>(base + 4 * t + align_up(sizeof(int64_t) * BH, kAlign));
+  uint8_t *ws = reinterpret_cast<uint8_t *>(dstatus) + align_up(sizeof(int) * kHostChunks, kAlign);
   const size_t ws_bytes = scratch_bytes - (ws - base);
-  if (cudaMemcpyAsync(dq, q, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess ||
-      cudaMemcpyAsync(dk, k, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess ||
-      cudaMemcpyAsync(dv, v, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess)
-    return SOLATTN_ECUDA;
-  solattn_stats stats{dkept, nullptr};
-  const int rf = solattn_forward(dq, dk, dv, dout, B, H, N, d, Bq, Bk, tau, mode, &stats, ws, ws_bytes, stream);
-  if (rf != SOLATTN_OK) return rf;
-  if (cudaMemcpyAsync(out, dout, bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess) return SOLATTN_ECUDA;
-  if (kept_per_head &&
-      cudaMemcpyAsync(kept_per_head, dkept, sizeof(int64_t) * B * H, cudaMemcpyDeviceToHost, st) != cudaSuccess)
-    return SOLATTN_ECUDA;
-  return solattn_get_status(ws, stream);
+
+  // Heads are independent, so the call runs as a pipeline over chunks of heads: the upload
+  // of chunk c+1 (stream `up`) and the download of chunk c-1 (stream `down`) overlap the
+  // forward of chunk c on the caller's stream. Every result equals the one-call result.
+  const int per = (BH + kHostChunks - 1) / kHostChunks;
+  const int nch = (BH + per - 1) / per;
+  const uint8_t *hq = static_cast<const uint8_t *>(q), *hk = static_cast<const uint8_t *>(k),
+                *hv = static_cast<const uint8_t *>(v);
+  uint8_t *hout = static_cast<uint8_t *>(out);
+  int rf = SOLATTN_OK;
+  bool enqueued = false;  // copies may be in flight on the pipe's streams
+  auto fail = [&](int code) {
+    if (enqueued) {  // the host buffers must outlive every copy that reads or writes them
+      cudaStreamSynchronize(hp->up);
+      cudaStreamSynchronize(hp->down);
+      cudaStreamSynchronize(st);
+    }
+    return code;
+  };
+  if (cudaEventRecord(hp->ev_start, st) != cudaSuccess || cudaStreamWaitEvent(hp->up, hp->ev_start, 0) != cudaSuccess)
+    return fail(SOLATTN_ECUDA);
+  for (int c = 0; c < nch; ++c) {
+    const int h0 = c * per, hn = (BH - h0 < per) ? BH - h0 : per;
+    const size_t off = head * h0, bytes = head * hn;
+    enqueued = true;
+    if (cudaMemcpyAsync(dq + off, hq + off, bytes, cudaMemcpyHostToDevice, hp->up) != cudaSuccess ||
+        cudaMemcpyAsync(dk + off, hk + off, bytes, cudaMemcpyHostToDevice, hp->up) != cudaSuccess ||
+        cudaMemcpyAsync(dv + off, hv + off, bytes, cudaMemcpyHostToDevice, hp->up) != cudaSuccess ||
+        cudaEventRecord(hp->ev_up[c], hp->up) != cudaSuccess || cudaStreamWaitEvent(st, hp->ev_up[c], 0) != cudaSuccess)
+      return fail(SOLATTN_ECUDA);
+    solattn_stats stats{dkept + h0, nullptr};
+    rf = solattn_forward(dq + off, dk + off, dv + off, dout + off, 1, hn, N, d, Bq, Bk, tau, mode, &stats, ws, ws_bytes,
+                         stream);
+    if (rf != SOLATTN_OK) return fail(rf);
+    // Each chunk clears the status word when it starts: keep this chunk's.
+    if (cudaMemcpyAsync(dstatus + c, ws + 4, sizeof(int), cudaMemcpyDeviceToDevice, st) != cudaSuccess ||
+        cudaEventRecord(hp->ev_done[c], st) != cudaSuccess ||
+        cudaStreamWaitEvent(hp->down, hp->ev_done[c], 0) != cudaSuccess ||
+        cudaMemcpyAsync(hout + off, dout + off, bytes, cudaMemcpyDeviceToHost, hp->down) != cudaSuccess)
+      return fail(SOLATTN_ECUDA);
+  }
+  int status[kHostChunks] = {};
+  if (cudaEventRecord(hp->ev_end, hp->down) != cudaSuccess || cudaStreamWaitEvent(st, hp->ev_end, 0) != cudaSuccess ||
+      (kept_per_head &&
+       cudaMemcpyAsync(kept_per_head, dkept, sizeof(int64_t) * BH, cudaMemcpyDeviceToHost, st) != cudaSuccess) ||
+      cudaMemcpyAsync(status, dstatus, sizeof(int) * nch, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return fail(SOLATTN_ECUDA);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return fail(SOLATTN_ECUDA);
+  for (int c = 0; c < nch; ++c)
+    if (status[c] != SOLATTN_OK) return status[c];
+  return SOLATTN_OK;
 }
 
 int solattn_watchdog_selftest(void *workspace, size_t ws_bytes, uint64_t limit_ns, void *stream) {

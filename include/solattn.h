@@ -38,10 +38,12 @@
  * solattn_forward_host, which synchronise the stream.
  *
  * Ownership: the caller allocates and owns every buffer (inputs, output,
- * statistics, workspace). The library allocates nothing at run time. Its one
+ * statistics, workspace). The library allocates no memory at run time. Its one
  * device-memory holding is the static scratch of solattn_forward_noalloc
  * (SOLATTN_NOALLOC_SCRATCH_BYTES), a module-scope device array that exists on
  * every GPU where the library's module is loaded, for the life of the process.
+ * solattn_forward_host also keeps, per device, two non-blocking copy streams and
+ * a few events, created at its first call there and kept for the process.
  */
 #ifndef SOLATTN_H
 #define SOLATTN_H
@@ -304,15 +306,26 @@ int solattn_route_topp(const float *qbar, const float *kbar, int B, int H, int N
 int solattn_get_status(const void *workspace, void *stream);
 
 /* Bytes of device scratch solattn_forward_host needs (device copies of q, k,
- * v, out, the per-head counts and the forward workspace). 0 if invalid. */
+ * v, out, the per-head counts, per-chunk status words and the forward
+ * workspace). 0 if invalid. */
 size_t solattn_host_workspace_size(int B, int H, int N, int d, int Bq, int Bk);
 
 /*
- * End-to-end call on HOST buffers: copies q, k, v (bf16 [B][H][N][d], host,
- * ideally pinned) to the device scratch, runs solattn_forward, copies the bf16
- * output to `out` and the per-head kept counts to `kept_per_head` (host int64
- * [B*H], may be NULL), then synchronises `stream` and returns the device status.
+ * End-to-end call on HOST buffers: copies q, k, v (bf16 [B][H][N][d], host) to
+ * the device scratch, runs the forward operator (running-max rule, `tau`,
+ * `mode` as in solattn_forward), copies the bf16 output to `out` and the
+ * per-head kept counts to `kept_per_head` (host int64 [B*H], may be NULL),
+ * synchronises `stream` and returns the first non-zero device status, else
+ * SOLATTN_OK.
+ * The (b, h) heads are independent, so the call is a pipeline over up to 16
+ * chunks of consecutive heads: the upload of one chunk and the download of the
+ * one before overlap the forward of the chunk between them. Uploads and
+ * downloads run on the library's copy streams for this device, the forward on
+ * `stream`; the result equals that of one solattn_forward over all heads.
+ * Copies overlap only from page-locked (pinned) host memory.
  * dev_scratch: device, 256-byte aligned, >= solattn_host_workspace_size(...).
+ * Calls on one device are serialised (they share the copy streams). On an error
+ * the call waits for the copies it issued before returning.
  */
 int solattn_forward_host(const void *q, const void *k, const void *v, void *out,
                          int B, int H, int N, int d, int Bq, int Bk, float tau, int mode,

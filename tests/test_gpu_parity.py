@@ -129,6 +129,34 @@ def test_host_entry_point_matches_device_call():
     assert torch.equal(kept, dev_kept)
 
 
+HOST_SHAPES = [
+    # (B, H, N, d, Bq, Bk, pinned): one head; 17 heads in 9 chunks with a one-head last
+    # chunk; 2 x 9 heads in 9 even chunks; 40 heads in 14 chunks; pageable host memory
+    (1, 1, 777, 128, 128, 128, True),
+    (1, 17, 1000, 128, 128, 64, True),
+    (2, 9, 700, 64, 64, 64, True),
+    (1, 40, 300, 128, 128, 128, True),
+    (1, 5, 900, 128, 128, 128, False),
+]
+
+
+@pytest.mark.parametrize("shape", HOST_SHAPES, ids=[str(s) for s in HOST_SHAPES])
+@pytest.mark.parametrize("mode", MODES)
+def test_pipelined_host_call_equals_one_device_call(shape, mode):
+    """The host entry point runs chunks of heads as a copy/compute pipeline; every
+    output element and kept count equals the one device call over all heads."""
+    from block_sparse_online_b200 import solattn
+    B, H, N, d, Bq, Bk, pinned = shape
+    q, k, v = synth.make_random(B, H, N, d, seed=100 + H)
+    dev_out, dev_kept, _ = run_gpu(q, k, v, Bq, Bk, 3.0, mode)
+    if pinned:
+        q, k, v = (t.pin_memory() for t in (q, k, v))
+    for _ in range(2):  # the second call reuses the device's copy streams and events
+        out, kept = solattn.solattn_forward_host(q, k, v, Bq, Bk, 3.0, mode)
+        assert torch.equal(out, dev_out)
+        assert torch.equal(kept, dev_kept)
+
+
 # ------------------------------------------------------------ full-size configurations
 
 def _full(name, taus, modes, per_head):
