@@ -96,6 +96,9 @@ struct FwdParams {
   // keep_correct with the block correction: per (b, h, query block), {M, L, -, -, C[D]}
   // (corr_stride floats), written by plan_kernel and read by the router.
   float *corr;
+  // Keep bits per (b, h, query block) ([BH][nQB][ceil(nKB/32)]), written by plan_kernel and
+  // read by the router; null in dense mode (no routing).
+  uint32_t *keep_bits;
 };
 
 // Floats per query block of the correction record: M (running proxy max, natural-log
@@ -390,13 +393,12 @@ template <class C>
 __device__ __forceinline__ void route_query_block(SmemCtl<C> &sc, RouteSlot<C> &rs, const FwdParams &p,
                                                   int bh, int sb, int qb, int lane) {
   constexpr int D = C::D;
-  constexpr int VPL = D / 32;
   const bool correct = (p.mode == 2) && !p.token_corr;  // block-level correction sums
-  float cacc[VPL];
-  float lacc, M;
-  // Keep decisions only: the correction sums of this query block were folded by the
-  // planning pass, through the same route_scan and hence the same decisions.
-  route_block<C::D, C::BQ, C::BK>(p, bh, qb, lane, false, sc.mask[sb], cacc, lacc, M);
+  // The planning pass routed this query block (route_block) and left its keep bits and,
+  // with the block correction, its correction record: the router only reads them.
+  const int nW = (p.nKB + 31) >> 5;
+  const uint32_t *kw = p.keep_bits + (static_cast<size_t>(bh) * p.nQB + qb) * nW;
+  for (int w = lane; w < nW; w += 32) sc.mask[sb][w] = kw[w];
   if (correct) {
     const float *rec = p.corr + (static_cast<size_t>(bh) * p.nQB + qb) * corr_stride<D>();
     for (int e = lane; e < D; e += 32) rs.Cv[sb][e] = __ldg(rec + 4 + e);
@@ -499,7 +501,8 @@ __device__ void run_router(SmemCtl<C> &sc, const FwdParams &p, int lane) {
       for (int w = lane; w < nW; w += 32) {
         const uint32_t word = sc.mask[sb][w];
         kept += __popc(word);
-        if (p.keep_mask) p.keep_mask[(static_cast<size_t>(bh) * p.nQB + qb) * nW + w] = word;
+        if (p.keep_mask && p.keep_mask != p.keep_bits)
+          p.keep_mask[(static_cast<size_t>(bh) * p.nQB + qb) * nW + w] = word;
       }
     }
 #pragma unroll
@@ -734,6 +737,10 @@ __device__ void run_mma(SmemCtl<C> &sc, const FwdParams &p, uint32_t tmem, uint8
     }
     if (!ok) break;
     if (first) {  // no P V for this warpgroup in this item (n == 1, w == 1)
+      // Arrive only once the previous item's epilogue is done, as a first P V would: this
+      // thread could otherwise run an item ahead of the other one and complete the previous
+      // item's o_full phase with two arrivals of its own, before the other's last P V.
+      if (!wait(&sc.o_empty, (o_it & 1) ^ 1)) break;
       mbar_arrive(&sc.o_full);
     } else {
       tc_commit(&sc.o_full);
@@ -1217,12 +1224,12 @@ __global__ void __launch_bounds__(256) gauss_theta_kernel(const float *qbar, con
 
 // ------------------------------------------------------------------ planning pass
 
-// Work-item schedule for the attention kernel. Each warp routes one item (query tile)
-// exactly as the kernel's router will and records how many key blocks the tile keeps
-// (its cost; the keep sets themselves do not leave the chip). In keep_correct with the
-// block correction it also folds every dropped block of each query block into the
-// correction record (p.corr: M, L and C, O(d) per query block), so that the attention
-// kernel's router only takes keep decisions. The last block to finish then orders the
+// Routing and work-item schedule for the attention kernel. Each warp routes one item
+// (query tile): it writes the keep bits of each query block (p.keep_bits, one bit per key
+// block; no proxy leaves the chip) and records how many key blocks the tile keeps (its
+// cost). In keep_correct with the block correction it also folds every dropped block of
+// each query block into the correction record (p.corr: M, L and C, O(d) per query block).
+// The attention kernel's router then only reads both. The last block to finish orders the
 // items: groups of `group_heads` consecutive heads in head order (the group's K/V stays
 // resident in L2), and within a group the costliest items first, so the short items
 // fill the end of the kernel instead of long ones starting late.
@@ -1250,6 +1257,9 @@ __global__ void __launch_bounds__(256) plan_kernel(const FwdParams p, int *cost,
       const int qb = tile * SUBQ + sb;
       if (qb >= p.nQB) continue;
       route_block<D, BQ, BK>(p, bh, qb, lane, correct, mask[warp][sb], cacc, lacc, M);
+      __syncwarp();
+      uint32_t *kw = p.keep_bits + (static_cast<size_t>(bh) * p.nQB + qb) * nW;
+      for (int w = lane; w < nW; w += 32) kw[w] = mask[warp][sb][w];
       if (correct) {
         float *rec = p.corr + (static_cast<size_t>(bh) * p.nQB + qb) * corr_stride<D>();
 #pragma unroll

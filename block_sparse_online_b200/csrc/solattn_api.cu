@@ -28,7 +28,7 @@ int nblocks(int N, int blk) { return (N + blk - 1) / blk; }
 bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 struct WsLayout {
-  size_t qbar, kbar, vbar, v16, cost, order, kmom, theta, kbar16, vbar16, corr, total;
+  size_t qbar, kbar, vbar, v16, cost, order, kmom, theta, kbar16, vbar16, corr, keep, total;
 };
 
 int check_shape(int B, int H, int N, int d, int Bq, int Bk) {
@@ -55,7 +55,8 @@ WsLayout ws_layout(int B, int H, int N, int d, int Bq, int Bk) {
   w.kbar16 = w.theta + align_up(bh * nblocks(N, Bq) * sizeof(float), kAlign);  // token-to-block correction
   w.vbar16 = w.kbar16 + align_up(bh * nblocks(N, Bk) * d * 2, kAlign);
   w.corr = w.vbar16 + align_up(bh * nblocks(N, Bk) * d * 2, kAlign);  // block correction per query block
-  w.total = w.corr + align_up(bh * nblocks(N, Bq) * (d + 4) * sizeof(float), kAlign);
+  w.keep = w.corr + align_up(bh * nblocks(N, Bq) * (d + 4) * sizeof(float), kAlign);  // keep bits
+  w.total = w.keep + align_up(bh * nblocks(N, Bq) * ((nblocks(N, Bk) + 31) / 32) * sizeof(uint32_t), kAlign);
   return w;
 }
 
@@ -375,6 +376,9 @@ int forward_impl(const void *q, const void *k, const void *v, void *out, int B, 
   p.token_corr = token ? 1 : 0;
   p.n_pseudo = token ? nblocks(nKB, Bk) : 0;
   p.corr = reinterpret_cast<float *>(ws + wl.corr);
+  // Keep bits: into the caller's keep mask when there is one (same layout), else scratch.
+  p.keep_bits = mode == SOLATTN_DENSE ? nullptr
+                                      : (stats->keep_mask ? stats->keep_mask : reinterpret_cast<uint32_t *>(ws + wl.keep));
   if (mode != SOLATTN_DENSE && rule != kRunningMax) {
     float *kmom = reinterpret_cast<float *>(ws + wl.kmom);
     float *theta = reinterpret_cast<float *>(ws + wl.theta);

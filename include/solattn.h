@@ -89,8 +89,10 @@ typedef struct {
 
 /*
  * Bytes of device workspace solattn_forward needs for this shape: a small
- * header (work counter, device status word), the pooled q, k, v blocks in fp32
- * and an fp16 copy of v. Returns 0 for an unsupported or invalid shape.
+ * header (work counter, device status word), the pooled q, k, v blocks in fp32,
+ * an fp16 copy of v, the work schedule, the keep bits and correction records of
+ * the routing pass, and what the Gaussian threshold and the token-to-block
+ * correction need. Returns 0 for an unsupported or invalid shape.
  */
 size_t solattn_workspace_size(int B, int H, int N, int d, int Bq, int Bk);
 

@@ -179,6 +179,29 @@ def test_video480_config():
     _full("video480", (2.0, 3.0, 4.0, 6.0, INF), MODES, per_head=32)
 
 
+def test_single_block_items_repeatable():
+    """Items that keep one key block leave the second softmax warpgroup without work, and
+    the routing-free attention kernel runs them back to back: the largest Gaussian
+    threshold (every query block keeps its top block only) and tau = 0 on the 480p shape.
+    Repeated calls give identical outputs, and sampled rows match the oracle."""
+    import dataclasses
+    cfg = dataclasses.replace(synth.CONFIGS["video480"], H=4)
+    q, k, v = synth.make_inputs(cfg)
+    blocks = sampled_blocks(cfg.B, cfg.H, cfg.N, cfg.Bq, cfg.Bk, 16, seed=cfg.seed + 7)
+    cases = [dict(tau=0.0, mode="keep_drop"), dict(tau=0.0, mode="keep_correct"),
+             dict(tau=0.0, mode="keep_drop", gauss=(INF, "exact"))]
+    for c in cases:
+        first = None
+        for _ in range(3):
+            out, kept, _ = run_gpu(q, k, v, cfg.Bq, cfg.Bk, c["tau"], c["mode"], gauss=c.get("gauss"))
+            if first is None:
+                first = (out, kept)
+            else:
+                assert torch.equal(out, first[0]) and torch.equal(kept, first[1]), c
+        check_case(q, k, v, cfg.Bq, cfg.Bk, c["tau"], c["mode"], qblocks=blocks, gauss=c.get("gauss"),
+                   label=f"single-block items {c}")
+
+
 @pytest.mark.slow
 def test_video720_config():
     _full("video720", (3.0, 4.0, 6.0), MODES, per_head=32)
