@@ -348,6 +348,32 @@ def quantiles(x):
             (("min", 0.0), ("p10", 0.1), ("p50", 0.5), ("p90", 0.9), ("max", 1.0))} | {"mean": round(float(x.mean()), 5)}
 
 
+# Spin of the GPU (clock cycles, ~10 ms) before a timed group of calls, so that the host's
+# enqueue latency does not show up as idle GPU time between the events.
+SPIN_CYCLES = 20_000_000
+
+
+def device_ms(fn, stream, reps=5, warm=2, rounds=3):
+    """Device time per call of `fn` in ms: `reps` back-to-back calls between two CUDA events
+    on `stream`, recorded behind a spin kernel that keeps the GPU busy while the host enqueues
+    them; the median over `rounds` groups, after `warm` untimed calls."""
+    import torch
+    for _ in range(warm):
+        fn()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(rounds):
+        torch.cuda._sleep(SPIN_CYCLES)
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for _ in range(reps):
+            fn()
+        a1.record(stream)
+        torch.cuda.synchronize()
+        ts.append(a0.elapsed_time(a1) / reps)
+    return statistics.median(ts)
+
+
 def config_sweep(name, dev, stream, peak_tf, reps=5):
     """One configuration: every (mode, tau) of its sweep timed as whole solattn_forward calls
     (median of `reps` after 2 warm-up calls), with keep ratios (block and token-weighted),
@@ -369,17 +395,7 @@ def config_sweep(name, dev, stream, peak_tf, reps=5):
     bq, bk = block_sizes(N, cfg.Bq), block_sizes(N, cfg.Bk)
 
     def timed(fn):
-        for _ in range(2):
-            fn()
-        ts = []
-        for _ in range(reps):
-            a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a0.record(stream)
-            fn()
-            a1.record(stream)
-            torch.cuda.synchronize()
-            ts.append(a0.elapsed_time(a1))
-        return statistics.median(ts)
+        return device_ms(fn, stream, reps=reps)
 
     dense_out, _, _ = solattn.solattn_forward(qd, kd, vd, cfg.Bq, cfg.Bk, 0.0, "dense", workspace=ws)
     dense_out = dense_out.float()
@@ -450,17 +466,7 @@ def routing_overhead(cfg, qd, kd, tau, stream):
                        device=qd.device)
 
     def timed(fn):
-        for _ in range(3):
-            fn()
-        ts = []
-        for _ in range(10):
-            a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a0.record(stream)
-            fn()
-            a1.record(stream)
-            torch.cuda.synchronize()
-            ts.append(a0.elapsed_time(a1))
-        return statistics.median(ts)
+        return device_ms(fn, stream, reps=10, warm=3)
 
     ours = timed(lambda: solattn.solattn_route_keep(qb, kb, N, cfg.Bq, cfg.Bk, tau, keep_mask=mask))
     topk = timed(lambda: solattn.solattn_route_topk(qb, kb, N, cfg.Bq, cfg.Bk, kk, keep_mask=mask, proxy_map=smap))
@@ -597,17 +603,8 @@ def main():
                 _, _, m = solattn.solattn_forward(qd, kd, vd, cfg.Bq, cfg.Bk, tau, mode, keep_mask=True, workspace=ws)
                 b = unpack(m, cfg.nKB)
                 ef = executed_flops(b, N, cfg.Bq, cfg.Bk, d)
-                ts = []
-                for i in range(8):
-                    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                    a0.record(stream)
-                    solattn.solattn_forward(qd, kd, vd, cfg.Bq, cfg.Bk, tau, mode, out=out, kept_per_head=kept,
-                                            workspace=ws)
-                    a1.record(stream)
-                    torch.cuda.synchronize()
-                    if i >= 3:
-                        ts.append(a0.elapsed_time(a1))
-                ms = statistics.median(ts)
+                ms = device_ms(lambda: solattn.solattn_forward(qd, kd, vd, cfg.Bq, cfg.Bk, tau, mode, out=out,
+                                                               kept_per_head=kept, workspace=ws), stream)
                 sweep.append({"mode": mode, "tau": None if math.isinf(tau) else tau, "ms": round(ms, 4),
                               "keep_ratio": round(float(b.mean()), 5),
                               "exec_tflops": round(ef / (ms * 1e-3) / 1e12, 2),
@@ -618,17 +615,9 @@ def main():
                                                  correction="token", keep_mask=True, workspace=ws)
             b = unpack(m, cfg.nKB)
             ef = executed_flops(b, N, cfg.Bq, cfg.Bk, d)
-            ts = []
-            for i in range(8):
-                a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                a0.record(stream)
-                solattn.solattn_forward_ex(qd, kd, vd, cfg.Bq, cfg.Bk, "keep_correct", tau=tau, correction="token",
-                                           out=out, kept_per_head=kept, workspace=ws)
-                a1.record(stream)
-                torch.cuda.synchronize()
-                if i >= 3:
-                    ts.append(a0.elapsed_time(a1))
-            ms = statistics.median(ts)
+            ms = device_ms(lambda: solattn.solattn_forward_ex(qd, kd, vd, cfg.Bq, cfg.Bk, "keep_correct", tau=tau,
+                                                              correction="token", out=out, kept_per_head=kept,
+                                                              workspace=ws), stream)
             sweep.append({"mode": "keep_correct", "correction": "token", "tau": tau, "ms": round(ms, 4),
                           "keep_ratio": round(float(b.mean()), 5),
                           "exec_tflops": round(ef / (ms * 1e-3) / 1e12, 2),
@@ -640,31 +629,15 @@ def main():
                                                            keep_mask=True, workspace=ws)
                 b = unpack(m, cfg.nKB)
                 ef = executed_flops(b, N, cfg.Bq, cfg.Bk, d)
-                ts = []
-                for i in range(8):
-                    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                    a0.record(stream)
-                    solattn.solattn_forward_gaussian(qd, kd, vd, cfg.Bq, cfg.Bk, beta, variant, "keep_correct",
-                                                     out=out, kept_per_head=kept, workspace=ws)
-                    a1.record(stream)
-                    torch.cuda.synchronize()
-                    if i >= 3:
-                        ts.append(a0.elapsed_time(a1))
-                ms = statistics.median(ts)
+                ms = device_ms(lambda: solattn.solattn_forward_gaussian(qd, kd, vd, cfg.Bq, cfg.Bk, beta, variant,
+                                                                        "keep_correct", out=out, kept_per_head=kept,
+                                                                        workspace=ws), stream)
                 sweep.append({"mode": "keep_correct", "threshold": f"gaussian-{variant}", "beta": beta,
                               "ms": round(ms, 4), "keep_ratio": round(float(b.mean()), 5),
                               "exec_tflops": round(ef / (ms * 1e-3) / 1e12, 2),
                               "dense_equiv_tflops": round(dense_flops / (ms * 1e-3) / 1e12, 2)})
-        ts = []
-        for i in range(6):
-            a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a0.record(stream)
-            solattn.solattn_forward(qd, kd, vd, cfg.Bq, cfg.Bk, 0.0, "dense", out=out, kept_per_head=kept, workspace=ws)
-            a1.record(stream)
-            torch.cuda.synchronize()
-            if i >= 2:
-                ts.append(a0.elapsed_time(a1))
-        ms = statistics.median(ts)
+        ms = device_ms(lambda: solattn.solattn_forward(qd, kd, vd, cfg.Bq, cfg.Bk, 0.0, "dense", out=out,
+                                                       kept_per_head=kept, workspace=ws), stream, reps=3)
         sweep.append({"mode": "dense", "tau": None, "ms": round(ms, 4), "keep_ratio": 1.0,
                       "exec_tflops": round(dense_flops / (ms * 1e-3) / 1e12, 2),
                       "dense_equiv_tflops": round(dense_flops / (ms * 1e-3) / 1e12, 2)})

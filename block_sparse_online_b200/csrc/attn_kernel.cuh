@@ -8,9 +8,9 @@
 //   warps 1, 3  MMA issuers (one thread each, for warpgroups A and B, taking turns):
 //               S = Q K_j^T into tensor memory (TMEM, bf16 -> fp32), O += P V_j with P
 //               read from TMEM (fp16 -> fp32).
-//   warp 2      router: on-the-fly block thresholding for the NEXT item (double-buffered),
-//               from the fp32 pooled blocks in L2; it picks up each query block's
-//               correction sums, which the planning pass folded (keep_correct).
+//   warp 2      router: for the NEXT item (double-buffered), reads the keep bits and the
+//               correction record the routing pass (plan_kernel) left for each query
+//               block, and builds the item's kept list in shared memory.
 //   warps 4..7  softmax warpgroup A, warps 8..11 softmax warpgroup B. The tile's kept
 //               list is split between them (A takes entries 0, 2, 4, ..., B takes 1, 3,
 //               5, ...); each keeps its own S, O, running max and sum for all 128 rows.
@@ -22,20 +22,19 @@
 //
 // Method (paperlayer summary "Sol-Attn: Accelerating Video Generation Inference
 // via On-the-Fly Attention Sparsification", §3 Methodology):
-//  * routing: block proxy s = mean(Q_i) . mean(K_j) / sqrt(d) is compared, as it is
-//    produced, against the running maximum of the proxies visited so far minus tau
-//    ("On-the-fly sparsification"); key blocks are visited from query block i's
-//    diagonal block upward with wrap-around. The kept list lives only in shared
-//    memory: no proxy map and no routing indices are written to HBM.
+//  * routing (plan_kernel, before this kernel): block proxy s = mean(Q_i) . mean(K_j) /
+//    sqrt(d) is compared, as it is produced, against the running maximum of the proxies
+//    visited so far minus tau ("On-the-fly sparsification"); key blocks are visited from
+//    query block i's diagonal block upward with wrap-around. The proxies stay in shared
+//    memory; only one keep bit per (query block, key block) reaches HBM.
 //  * exact attention on kept blocks with one online-softmax state per row
 //    ("Unified execution": one online-softmax state, original K/V tiles loaded only
 //    for routed indices).
 //  * each dropped block re-enters as one pseudo-key of weight n_j e^{s} and value
 //    mean(V_j) ("Approximate correction": zeroth-order proxy-score reuse with pooled
 //    keys and summed values). Because s does not depend on the query row, the
-//    correction is one d-vector and one scalar per query block. The planning pass
-//    (plan_kernel), which routes every query tile before this kernel, folds it with the
-//    whole GPU's parallelism; the router here only takes the keep decisions.
+//    correction is one d-vector and one scalar per query block, which the routing pass
+//    folds with the whole GPU's parallelism.
 #pragma once
 
 #include <cstdint>
@@ -192,210 +191,13 @@ __device__ __forceinline__ float u2f(uint32_t x) { return __uint_as_float(x); }
 
 // ------------------------------------------------------------------ router
 
-// Warp transpose-sum: every lane holds 32 partial values v[0..31]; on return lane l
-// holds the sum over the 32 lanes of v[l]. A butterfly of 31 shuffles (16 + 8 + 4 + 2
-// + 1): at each stage a lane keeps the half of its values whose index bit matches its
-// own lane bit and adds the partner's copy of that half.
-__device__ __forceinline__ float warp_transpose_sum32(float (&v)[32], int lane) {
-#pragma unroll
-  for (int w = 16; w >= 1; w >>= 1) {
-    const bool hi = (lane & w) != 0;
-#pragma unroll
-    for (int i = 0; i < w; ++i) {
-      const float keep = hi ? v[i + w] : v[i];
-      const float send = hi ? v[i] : v[i + w];
-      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, w);
-    }
-  }
-  return v[0];
-}
-
-template <int VPL>
-struct VecOf;
-template <>
-struct VecOf<4> {
-  using T = float4;
-  static __device__ __forceinline__ float dot(const float (&a)[4], const float4 &b) {
-    return fmaf(a[3], b.w, fmaf(a[2], b.z, fmaf(a[1], b.y, a[0] * b.x)));
-  }
-  static __device__ __forceinline__ void axpy(float (&acc)[4], float w, const float4 &b) {
-    acc[0] = fmaf(w, b.x, acc[0]);
-    acc[1] = fmaf(w, b.y, acc[1]);
-    acc[2] = fmaf(w, b.z, acc[2]);
-    acc[3] = fmaf(w, b.w, acc[3]);
-  }
-  static __device__ __forceinline__ float4 zero() { return make_float4(0.f, 0.f, 0.f, 0.f); }
-};
-template <>
-struct VecOf<2> {
-  using T = float2;
-  static __device__ __forceinline__ float dot(const float (&a)[2], const float2 &b) {
-    return fmaf(a[1], b.y, a[0] * b.x);
-  }
-  static __device__ __forceinline__ void axpy(float (&acc)[2], float w, const float2 &b) {
-    acc[0] = fmaf(w, b.x, acc[0]);
-    acc[1] = fmaf(w, b.y, acc[1]);
-  }
-  static __device__ __forceinline__ float2 zero() { return make_float2(0.f, 0.f); }
-};
-
-// Route one query block: visit its key blocks in order, keep those whose proxy clears
-// the running maximum minus tau, and (if `correct`) fold every dropped block into the
-// correction sums (cacc, lacc relative to the running max M). Keep bits are OR-ed into
-// `msk` (shared memory, zeroed by the caller). Lane-per-dimension layout: each pooled
-// row is one coalesced 128/256-byte load across the warp, loads are issued 8 rows at a
-// time, and the 32 per-block dot products of a chunk are finished with one
-// transpose-sum. The attention kernel's router and the planning kernel both route
-// through this function, so they take identical decisions.
-// Routes query block qb: sets the keep bits in msk and, when `correct`, accumulates the
-// correction of the dropped blocks. Returns the number of kept blocks; top_j receives the
-// block with the largest proxy (lowest index on ties; Gaussian threshold only), and
-// force_j (>= 0) is kept whatever its proxy.
-template <int D, int BQ, int BK>
-__device__ __forceinline__ int route_scan(const FwdParams &p, int bh, int qb, int lane, bool correct, uint32_t *msk,
-                                          float (&cacc)[D / 32], float &lacc, float &M, int force_j, int &top_j) {
-  constexpr int VPL = D / 32;  // dimensions per lane
-  using V = VecOf<VPL>;
-  using VecT = typename V::T;
-  constexpr int G = 8;  // rows in flight per lane
-  const int nKB = p.nKB;
-  const float inv_sqrt_d = rsqrtf(static_cast<float>(D));
-  const int j0 = min((qb * BQ) / BK, nKB - 1);
-  const VecT *kb = reinterpret_cast<const VecT *>(p.kbar + static_cast<size_t>(bh) * nKB * D) + lane;
-  const VecT *vb = reinterpret_cast<const VecT *>(p.vbar + static_cast<size_t>(bh) * nKB * D) + lane;
-
-  float qv[VPL];
-  {
-    const float *qr = p.qbar + (static_cast<size_t>(bh) * p.nQB + qb) * D + lane * VPL;
-#pragma unroll
-    for (int e = 0; e < VPL; ++e) qv[e] = __ldg(qr + e);
-  }
-  M = -CUDART_INF_F;
-#pragma unroll
-  for (int e = 0; e < VPL; ++e) cacc[e] = 0.f;
-  lacc = 0.f;
-  const bool gauss = p.theta != nullptr;
-  const float th = gauss ? __ldg(p.theta + static_cast<size_t>(bh) * p.nQB + qb) : 0.f;
-  const int nsb = p.n_sink_blocks;  // sink blocks are kept outright
-  int kept = 0;
-  float top_s = -CUDART_INF_F;
-  top_j = nKB;
-
-  for (int t0 = 0; t0 < nKB; t0 += 32) {
-    float part[32];
-#pragma unroll
-    for (int g = 0; g < 32 / G; ++g) {
-      VecT kx[G];
-#pragma unroll
-      for (int e = 0; e < G; ++e) {
-        const int t = t0 + g * G + e;
-        int j = j0 + t;
-        if (j >= nKB) j -= nKB;
-        kx[e] = (t < nKB) ? __ldg(kb + static_cast<size_t>(j) * 32) : V::zero();
-      }
-#pragma unroll
-      for (int e = 0; e < G; ++e) part[g * G + e] = V::dot(qv, kx[e]);
-    }
-    const int tt = t0 + lane;
-    const bool valid = tt < nKB;
-    int j = j0 + tt;
-    if (j >= nKB) j -= nKB;
-    if (!valid) j = 0;
-    float s = warp_transpose_sum32(part, lane) * inv_sqrt_d;
-    if (!valid) s = -CUDART_INF_F;
-    // Running maximum in visit order: inclusive prefix max over the lanes.
-    float m = s;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const float y = __shfl_up_sync(0xffffffffu, m, off);
-      if (lane >= off) m = fmaxf(m, y);
-    }
-    m = fmaxf(m, M);
-    const float thr = gauss ? th : m - p.tau;
-    const bool keep = valid && (s >= thr || j == force_j || j < nsb);
-    const float Mn = __shfl_sync(0xffffffffu, m, 31);
-    if (keep) atomicOr(&msk[j >> 5], 1u << (j & 31));
-    kept += __popc(__ballot_sync(0xffffffffu, keep));
-    if (gauss) {
-      float bs = valid ? s : -CUDART_INF_F;
-      int bj = valid ? j : nKB;
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        const float os = __shfl_xor_sync(0xffffffffu, bs, off);
-        const int oj = __shfl_xor_sync(0xffffffffu, bj, off);
-        if (os > bs || (os == bs && oj < bj)) {
-          bs = os;
-          bj = oj;
-        }
-      }
-      if (bs > top_s || (bs == top_s && bj < top_j)) {
-        top_s = bs;
-        top_j = bj;
-      }
-    }
-    if (correct) {
-      if (Mn > M) {
-        const float f = expf(M - Mn);  // 0 on the first chunk (M = -inf)
-#pragma unroll
-        for (int e = 0; e < VPL; ++e) cacc[e] *= f;
-        lacc *= f;
-        M = Mn;
-      }
-      const bool drop = valid && !keep;
-      const float nj = (j == nKB - 1) ? static_cast<float>(p.N - j * BK) : static_cast<float>(BK);
-      const float w = drop ? nj * expf(s - M) : 0.f;
-      lacc += w;
-      uint32_t dm = __ballot_sync(0xffffffffu, drop);
-      while (dm) {  // dm is warp-uniform
-        int src[G];
-#pragma unroll
-        for (int e = 0; e < G; ++e) {
-          src[e] = dm ? (__ffs(dm) - 1) : -1;
-          dm = dm ? (dm & (dm - 1)) : 0u;
-        }
-        VecT vx[G];
-        float wb[G];
-#pragma unroll
-        for (int e = 0; e < G; ++e) {
-          const int b = src[e] < 0 ? 0 : src[e];
-          const int jb = __shfl_sync(0xffffffffu, j, b);
-          wb[e] = src[e] < 0 ? 0.f : __shfl_sync(0xffffffffu, w, b);
-          vx[e] = src[e] < 0 ? V::zero() : __ldg(vb + static_cast<size_t>(jb) * 32);
-        }
-#pragma unroll
-        for (int e = 0; e < G; ++e) V::axpy(cacc, wb[e], vx[e]);
-      }
-    } else {
-      M = Mn;
-    }
-  }
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) lacc += __shfl_xor_sync(0xffffffffu, lacc, off);
-  return kept;
-}
-
-// route_scan under either rule. Under the Gaussian threshold a query block whose proxies
-// all fall below its threshold keeps its top block: the scan is repeated with that block
-// forced (the correction sums of the first scan included it as dropped).
-template <int D, int BQ, int BK>
-__device__ __forceinline__ int route_block(const FwdParams &p, int bh, int qb, int lane, bool correct, uint32_t *msk,
-                                           float (&cacc)[D / 32], float &lacc, float &M) {
-  int top_j = 0;
-  int kept = route_scan<D, BQ, BK>(p, bh, qb, lane, correct, msk, cacc, lacc, M, -1, top_j);
-  if (p.theta && kept == 0) {
-    int unused = 0;
-    kept = route_scan<D, BQ, BK>(p, bh, qb, lane, correct, msk, cacc, lacc, M, top_j, unused);
-  }
-  return kept;
-}
-
 template <class C>
 __device__ __forceinline__ void route_query_block(SmemCtl<C> &sc, RouteSlot<C> &rs, const FwdParams &p,
                                                   int bh, int sb, int qb, int lane) {
   constexpr int D = C::D;
   const bool correct = (p.mode == 2) && !p.token_corr;  // block-level correction sums
-  // The planning pass routed this query block (route_block) and left its keep bits and,
-  // with the block correction, its correction record: the router only reads them.
+  // The routing pass (plan_kernel) left this query block's keep bits and, with the block
+  // correction, its correction record: the router only reads them.
   const int nW = (p.nKB + 31) >> 5;
   const uint32_t *kw = p.keep_bits + (static_cast<size_t>(bh) * p.nQB + qb) * nW;
   for (int w = lane; w < nW; w += 32) sc.mask[sb][w] = kw[w];
@@ -1219,118 +1021,6 @@ __global__ void __launch_bounds__(256) gauss_theta_kernel(const float *qbar, con
     else if (beta == CUDART_INF_F) t = CUDART_INF_F;
     else t = mu * rsqrtf(static_cast<float>(D)) + beta * sqrtf(fmaxf(var / static_cast<float>(D), 0.f));
     theta[static_cast<size_t>(bh) * nQB + i] = t;
-  }
-}
-
-// ------------------------------------------------------------------ planning pass
-
-// Routing and work-item schedule for the attention kernel. Each warp routes one item
-// (query tile): it writes the keep bits of each query block (p.keep_bits, one bit per key
-// block; no proxy leaves the chip) and records how many key blocks the tile keeps (its
-// cost). In keep_correct with the block correction it also folds every dropped block of
-// each query block into the correction record (p.corr: M, L and C, O(d) per query block).
-// The attention kernel's router then only reads both. The last block to finish orders the
-// items: groups of `group_heads` consecutive heads in head order (the group's K/V stays
-// resident in L2), and within a group the costliest items first, so the short items
-// fill the end of the kernel instead of long ones starting late.
-template <int D, int BQ, int BK, int SUBQ>
-__global__ void __launch_bounds__(256) plan_kernel(const FwdParams p, int *cost, int *order, unsigned int *done,
-                                                   int group_heads) {
-  constexpr int WARPS = 8;
-  __shared__ uint32_t mask[WARPS][SUBQ][kMaskWords];
-  __shared__ int hist[kMaxKeyBlocks + 2];
-  __shared__ int warp_tot[WARPS];
-  __shared__ int is_last;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nW = (p.nKB + 31) >> 5;
-  const int item = blockIdx.x * WARPS + warp;
-  if (item < p.n_items) {
-    const int bh = item / p.items_per_head;
-    const int tile = item - bh * p.items_per_head;
-    for (int sb = 0; sb < SUBQ; ++sb)
-      for (int w = lane; w < nW; w += 32) mask[warp][sb][w] = 0u;
-    __syncwarp();
-    float cacc[D / 32];
-    float lacc, M;
-    const bool correct = (p.mode == 2) && !p.token_corr;
-    for (int sb = 0; sb < SUBQ; ++sb) {
-      const int qb = tile * SUBQ + sb;
-      if (qb >= p.nQB) continue;
-      route_block<D, BQ, BK>(p, bh, qb, lane, correct, mask[warp][sb], cacc, lacc, M);
-      __syncwarp();
-      uint32_t *kw = p.keep_bits + (static_cast<size_t>(bh) * p.nQB + qb) * nW;
-      for (int w = lane; w < nW; w += 32) kw[w] = mask[warp][sb][w];
-      if (correct) {
-        float *rec = p.corr + (static_cast<size_t>(bh) * p.nQB + qb) * corr_stride<D>();
-#pragma unroll
-        for (int e = 0; e < D / 32; ++e) rec[4 + lane * (D / 32) + e] = cacc[e];
-        if (lane == 0) {
-          rec[0] = M;
-          rec[1] = lacc;
-        }
-      }
-    }
-    __syncwarp();
-    int cnt = 0;
-    for (int w = lane; w < nW; w += 32) {
-      uint32_t u = 0;
-      for (int sb = 0; sb < SUBQ; ++sb) u |= mask[warp][sb][w];
-      cnt += __popc(u);
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, off);
-    if (lane == 0) cost[item] = cnt;
-  }
-  // The last block to finish builds the order.
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) is_last = (atomicAdd(done, 1u) == gridDim.x - 1);
-  __syncthreads();
-  if (!is_last) return;
-  __threadfence();
-  const int BH = p.n_items / p.items_per_head;
-  const int nbins = p.nKB + 1;  // cost in [0, nKB]
-  for (int h0 = 0; h0 < BH; h0 += group_heads) {
-    const int i0 = h0 * p.items_per_head;
-    const int i1 = min(BH, h0 + group_heads) * p.items_per_head;
-    for (int c = threadIdx.x; c < nbins; c += blockDim.x) hist[c] = 0;
-    __syncthreads();
-    for (int i = i0 + threadIdx.x; i < i1; i += blockDim.x) atomicAdd(&hist[cost[i]], 1);
-    __syncthreads();
-    // Exclusive scan over descending cost: start[c] = number of items costlier than c.
-    // Each thread owns a contiguous run of bins (from the costliest end).
-    const int per = (nbins + blockDim.x - 1) / blockDim.x;
-    const int c_hi = nbins - 1 - threadIdx.x * per;  // this thread's bins: c_hi, c_hi-1, ...
-    int local = 0;
-    for (int k = 0; k < per; ++k) {
-      const int c = c_hi - k;
-      if (c >= 0) local += hist[c];
-    }
-    int incl = local;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, incl, off);
-      if (lane >= off) incl += y;
-    }
-    if (lane == 31) warp_tot[warp] = incl;
-    __syncthreads();
-    int before = 0;
-    for (int w = 0; w < warp; ++w) before += warp_tot[w];
-    int run = before + incl - local;
-    for (int k = 0; k < per; ++k) {
-      const int c = c_hi - k;
-      if (c >= 0) {
-        const int cnt_c = hist[c];
-        hist[c] = run;
-        run += cnt_c;
-      }
-    }
-    __syncthreads();
-    for (int i = i0 + threadIdx.x; i < i1; i += blockDim.x) {
-      const int pos = atomicAdd(&hist[cost[i]], 1);
-      order[i0 + pos] = i;
-    }
-    __syncthreads();
   }
 }
 

@@ -4,9 +4,10 @@
 // routing that consumes the proxy scores on chip against top-k and top-p routing, which
 // materialise the proxy map and traverse whole rows of it; §2 Block-Sparse Attention).
 //
-//   route_kernel      Sol-Attn's running-max rule: each warp streams one query block's
-//                     pooled keys through route_scan (the attention kernel's router) and
-//                     writes only the keep bits. No proxy leaves the chip.
+//   plan_kernel       (plan_kernel.cuh) Sol-Attn's running-max rule, the forward's own
+//                     routing pass with its correction and schedule steps off: proxies of
+//                     a group of query blocks in shared memory, keep bits out. No proxy
+//                     leaves the chip.
 //   proxy_map_kernel  s_ij = q_i . k_j / sqrt(d) for every (query block, key block), to HBM.
 //   select_kernel     one CTA per proxy row: a bitonic sort of the row in shared memory,
 //                     then top-k (the k largest proxies) or top-p (the heaviest blocks,
@@ -16,29 +17,9 @@
 
 #include <cstdint>
 
-#include "attn_kernel.cuh"
+#include "plan_kernel.cuh"
 
 namespace solattn {
-
-// One warp per (b, h, query block) row of the proxy map.
-template <int D, int BQ, int BK>
-__global__ void __launch_bounds__(256) route_kernel(const FwdParams p, uint32_t *keep_mask, int n_rows) {
-  constexpr int WARPS = 8;
-  __shared__ uint32_t mask[WARPS][kMaskWords];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int r = blockIdx.x * WARPS + warp;
-  if (r >= n_rows) return;  // warp-uniform
-  const int bh = r / p.nQB;
-  const int qb = r - bh * p.nQB;
-  const int nW = (p.nKB + 31) >> 5;
-  for (int w = lane; w < nW; w += 32) mask[warp][w] = 0u;
-  __syncwarp();
-  float cacc[D / 32];
-  float lacc, M;
-  route_block<D, BQ, BK>(p, bh, qb, lane, false, mask[warp], cacc, lacc, M);
-  __syncwarp();
-  for (int w = lane; w < nW; w += 32) keep_mask[static_cast<size_t>(r) * nW + w] = mask[warp][w];
-}
 
 // smap[bh][i][j] = qbar[bh][i] . kbar[bh][j] / sqrt(D) in fp32. Grid (ceil(nKB / 64),
 // ceil(nQB / 64), B*H), 256 threads, each a 4 x 4 block of outputs; 64-row tiles of the

@@ -9,6 +9,7 @@
 #include <mutex>
 
 #include "attn_kernel.cuh"
+#include "plan_kernel.cuh"
 #include "pool_kernel.cuh"
 #include "route_kernels.cuh"
 #include "solattn.h"
@@ -164,26 +165,42 @@ int dispatch_tiles(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorM
   return launch_fwd<C>(mq, mk, mv, mkp, mvp, p, sms, st);
 }
 
+// The routing pass over B*H heads. cost == null: keep bits only (the routing-only entry
+// point); otherwise also the correction records (keep_correct) and the work order.
 template <int D, int BK, int SUBQ>
-int launch_plan(const FwdParams &p, int *cost, int *order, unsigned int *done, int group_heads, cudaStream_t st) {
-  const int grid = (p.n_items + 7) / 8;
-  plan_kernel<D, 128 / SUBQ, BK, SUBQ><<<grid, 256, 0, st>>>(p, cost, order, done, group_heads);
+int launch_plan(const FwdParams &p, int BH, uint32_t *keep_out, int *cost, int *order, unsigned int *done,
+                int group_heads, cudaStream_t st) {
+  auto kern = plan_kernel<D, 128 / SUBQ, BK, SUBQ>;
+  static bool attr_set[64] = {};  // per device; guarded by g_mu
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return SOLATTN_ECUDA;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!attr_set[dev]) {
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(plan_smem_bytes<D>(kMaxKeyBlocks))) != cudaSuccess)
+        return SOLATTN_ECUDA;
+      attr_set[dev] = true;
+    }
+  }
+  const dim3 grid((p.nQB + kPlanQG - 1) / kPlanQG, BH);
+  kern<<<grid, kPlanWarps * 32, plan_smem_bytes<D>(p.nKB), st>>>(p, keep_out, cost, order, done, group_heads);
   return cudaGetLastError() == cudaSuccess ? SOLATTN_OK : SOLATTN_ECUDA;
 }
 
-int dispatch_plan(int d, int Bq, int Bk, const FwdParams &p, int *cost, int *order, unsigned int *done,
-                  int group_heads, cudaStream_t st) {
+int dispatch_plan(int d, int Bq, int Bk, const FwdParams &p, int BH, uint32_t *keep_out, int *cost, int *order,
+                  unsigned int *done, int group_heads, cudaStream_t st) {
   const int subq = 128 / Bq;
   if (d == 128) {
-    if (Bk == 128) return subq == 1 ? launch_plan<128, 128, 1>(p, cost, order, done, group_heads, st)
-                                    : launch_plan<128, 128, 2>(p, cost, order, done, group_heads, st);
-    return subq == 1 ? launch_plan<128, 64, 1>(p, cost, order, done, group_heads, st)
-                     : launch_plan<128, 64, 2>(p, cost, order, done, group_heads, st);
+    if (Bk == 128) return subq == 1 ? launch_plan<128, 128, 1>(p, BH, keep_out, cost, order, done, group_heads, st)
+                                    : launch_plan<128, 128, 2>(p, BH, keep_out, cost, order, done, group_heads, st);
+    return subq == 1 ? launch_plan<128, 64, 1>(p, BH, keep_out, cost, order, done, group_heads, st)
+                     : launch_plan<128, 64, 2>(p, BH, keep_out, cost, order, done, group_heads, st);
   }
-  if (Bk == 128) return subq == 1 ? launch_plan<64, 128, 1>(p, cost, order, done, group_heads, st)
-                                  : launch_plan<64, 128, 2>(p, cost, order, done, group_heads, st);
-  return subq == 1 ? launch_plan<64, 64, 1>(p, cost, order, done, group_heads, st)
-                   : launch_plan<64, 64, 2>(p, cost, order, done, group_heads, st);
+  if (Bk == 128) return subq == 1 ? launch_plan<64, 128, 1>(p, BH, keep_out, cost, order, done, group_heads, st)
+                                  : launch_plan<64, 128, 2>(p, BH, keep_out, cost, order, done, group_heads, st);
+  return subq == 1 ? launch_plan<64, 64, 1>(p, BH, keep_out, cost, order, done, group_heads, st)
+                   : launch_plan<64, 64, 2>(p, BH, keep_out, cost, order, done, group_heads, st);
 }
 
 int dispatch(int d, int Bq, int Bk, const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
@@ -392,10 +409,15 @@ int forward_impl(const void *q, const void *k, const void *v, void *out, int B, 
     const size_t head_kv = static_cast<size_t>(N) * d * 4;
     int group_heads = static_cast<int>((64ull << 20) / (head_kv ? head_kv : 1));
     group_heads = group_heads < 1 ? 1 : (group_heads > BH ? BH : group_heads);
+    // The routing pass orders a group's items in shared memory: at most kPlanOrderCap of
+    // them (or one head's, up to 1024).
+    const int per_head = items_total(1, 1, N);
+    if (group_heads > 1 && group_heads * per_head > kPlanOrderCap)
+      group_heads = kPlanOrderCap / per_head > 1 ? kPlanOrderCap / per_head : 1;
     int *cost = reinterpret_cast<int *>(ws + wl.cost);
     int *order = reinterpret_cast<int *>(ws + wl.order);
-    const int rp = dispatch_plan(d, Bq, Bk, p, cost, order, reinterpret_cast<unsigned int *>(ws + 8), group_heads,
-                                 st);
+    const int rp = dispatch_plan(d, Bq, Bk, p, BH, p.keep_bits, cost, order, reinterpret_cast<unsigned int *>(ws + 8),
+                                 group_heads, st);
     if (rp != SOLATTN_OK) return rp;
     p.order = order;
   }
@@ -409,23 +431,6 @@ int forward_impl(const void *q, const void *k, const void *v, void *out, int B, 
 }
 
 // ---- routing on its own (routing-overhead measurement)
-
-template <int D, int BQ, int BK>
-int launch_route_t(const FwdParams &p, uint32_t *mask, int n_rows, cudaStream_t st) {
-  route_kernel<D, BQ, BK><<<(n_rows + 7) / 8, 256, 0, st>>>(p, mask, n_rows);
-  return cudaGetLastError() == cudaSuccess ? SOLATTN_OK : SOLATTN_ECUDA;
-}
-
-int launch_route(int d, int Bq, int Bk, const FwdParams &p, uint32_t *mask, int n_rows, cudaStream_t st) {
-  if (d == 128) {
-    if (Bq == 128) return Bk == 128 ? launch_route_t<128, 128, 128>(p, mask, n_rows, st)
-                                    : launch_route_t<128, 128, 64>(p, mask, n_rows, st);
-    return Bk == 128 ? launch_route_t<128, 64, 128>(p, mask, n_rows, st) : launch_route_t<128, 64, 64>(p, mask, n_rows, st);
-  }
-  if (Bq == 128) return Bk == 128 ? launch_route_t<64, 128, 128>(p, mask, n_rows, st)
-                                  : launch_route_t<64, 128, 64>(p, mask, n_rows, st);
-  return Bk == 128 ? launch_route_t<64, 64, 128>(p, mask, n_rows, st) : launch_route_t<64, 64, 64>(p, mask, n_rows, st);
-}
 
 template <int P>
 int launch_select_t(const float *smap, uint32_t *mask, int rows, int nKB, int N, int Bk, int topp, int k, float pm,
@@ -707,8 +712,9 @@ int solattn_route_keep(const float *qbar, const float *kbar, int B, int H, int N
   p.tau = tau;
   p.qbar = qbar;
   p.kbar = kbar;
-  const int rows = B * H * p.nQB;
-  return launch_route(d, Bq, Bk, p, keep_mask, rows, static_cast<cudaStream_t>(stream));
+  // The forward's routing pass with its correction and schedule steps off (cost = null).
+  return dispatch_plan(d, Bq, Bk, p, B * H, keep_mask, nullptr, nullptr, nullptr, 1,
+                       static_cast<cudaStream_t>(stream));
 }
 
 size_t solattn_proxy_map_bytes(int B, int H, int N, int Bq, int Bk) {
