@@ -1,6 +1,6 @@
 """Build libsolattn.so (sm_100a) in-tree with nvcc.
 
-    python -m block_sparse_online_b200.build [--verbose]
+    python -m block_sparse_online_b200.build [--verbose] [--debug]
 
 The library is written next to this file so that it travels with the source
 tree; the Python binding loads it from there.
@@ -17,6 +17,10 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libsolattn.so")
+# The same library with the kernels' device-side bounds checks compiled in (-DSOLATTN_DEBUG):
+# a failed check records SOLATTN_EBOUNDS in the workspace status word instead of touching
+# memory out of range. Same exports; load it explicitly (solattn.load_library(DEBUG_LIB)).
+DEBUG_LIB = os.path.join(PKG, "libsolattn_debug.so")
 SOURCES = ["solattn_api.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
@@ -28,9 +32,12 @@ def nvcc() -> str:
     raise RuntimeError("nvcc not found")
 
 
-def build(verbose: bool = False, extra=()) -> str:
+def build(verbose: bool = False, extra=(), debug: bool = False) -> str:
+    out = DEBUG_LIB if debug else LIB
     cmd = [nvcc(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "-shared", "-Xcompiler", "-fPIC",
-           "-I", INCLUDE, "-I", CSRC, "-o", LIB, *[os.path.join(CSRC, s) for s in SOURCES], *extra]
+           "-I", INCLUDE, "-I", CSRC, "-o", out, *[os.path.join(CSRC, s) for s in SOURCES], *extra]
+    if debug:
+        cmd.insert(1, "-DSOLATTN_DEBUG")
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
     res = subprocess.run(cmd, capture_output=True, text=True)
@@ -38,8 +45,8 @@ def build(verbose: bool = False, extra=()) -> str:
         raise RuntimeError("nvcc failed:\n" + res.stdout + res.stderr)
     if verbose:
         sys.stdout.write(res.stdout + res.stderr)
-    return LIB
+    return out
 
 
 if __name__ == "__main__":
-    print(build(verbose="--verbose" in sys.argv))
+    print(build(verbose="--verbose" in sys.argv, debug="--debug" in sys.argv))

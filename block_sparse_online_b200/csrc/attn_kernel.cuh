@@ -55,10 +55,15 @@ constexpr int kMaskWords = kMaxKeyBlocks / 32;
 constexpr int kPseudoFlag = 0x8000;
 constexpr int kMaxPseudo = kMaxKeyBlocks / 64;
 constexpr int kStatusTimeout = -4;
+constexpr int kStatusBounds = -6;  // a debug-build bounds check failed
 constexpr float kLog2e = 1.4426950408889634f;
 // Lazy rescaling: a row's reference max moves only when the tile max exceeds it by
-// more than this many log2 units, so P stays <= 2^8 and O is rarely rescaled.
+// more than this many log2 units, so O is rarely rescaled (P <= 2^8 on the tile that moves
+// it; a lagging reference is kept while every row sum of a tile stays <= 2^15).
 constexpr float kRescaleSlack = 8.0f;
+// Largest row sum of a tile exponentiated against a reference max that may lag the row:
+// every value is then <= 2^15, inside fp16's range.
+constexpr float kSpecRowSumLimit = 32768.0f;
 // Pairs of exponentials computed on the FMA pipe (polynomial) instead of the MUFU unit:
 // bit e % 8 of this mask set -> pair e of a 16-pair chunk goes to the polynomial.
 constexpr uint32_t kPolyMask = 0x80u;
@@ -136,7 +141,7 @@ struct Cfg {
   static constexpr int CTRL_REGS = 120;
   static constexpr int SOFTMAX_REGS = 192;
   static_assert(128 * CTRL_REGS + 256 * SOFTMAX_REGS <= 384 * 168, "register split");
-  // S = Q K^T in bf16; O += P V in fp16 (P in [0, 2^8] after the lazy rescale; V is the
+  // S = Q K^T in bf16; O += P V in fp16 (P in [0, 2^15] under the lazy rescale; V is the
   // fp16 copy written by the pooling pass).
   static constexpr uint32_t IDESC_QK = idesc_16bit_f32(128, BK, false, false);
   static constexpr uint32_t IDESC_PV = idesc_16bit_f32(128, D, true, true);
@@ -182,10 +187,36 @@ constexpr size_t fwd_smem_bytes() {
          static_cast<size_t>(C::NSLOT) * C::KV_BYTES + sizeof(SmemCtl<C>);
 }
 
+// The first error of a launch is kept: a role that gave up on a wait records a timeout
+// unless another role recorded an error first, then raises the block-wide abort flag.
 __device__ __forceinline__ void raise_abort(int *abort_flag, int *status) {
-  atomicExch(status, kStatusTimeout);
+  atomicCAS(status, 0, kStatusTimeout);
   *reinterpret_cast<volatile int *>(abort_flag) = 1;
 }
+
+// Debug builds (-DSOLATTN_DEBUG) check the indices each role derives from shared state
+// before it uses them for a copy, an MMA operand or a store. A failed check records
+// kStatusBounds (if no error is recorded yet) and raises the abort flag; the role then
+// leaves as it does after a timeout, and the other roles follow at their next wait.
+// Release builds compile every check to `true`.
+__device__ __forceinline__ bool debug_fail(int *abort_flag, int *status) {
+  atomicCAS(status, 0, kStatusBounds);
+  *reinterpret_cast<volatile int *>(abort_flag) = 1;
+  return false;
+}
+// Kernels without an abort flag (the routing pass) record the status only; the routing-only
+// entry point runs without a status word (null), and then a failed check only skips the access.
+__device__ __forceinline__ bool debug_fail_status(int *status) {
+  if (status) atomicCAS(status, 0, kStatusBounds);
+  return false;
+}
+#ifdef SOLATTN_DEBUG
+#define SOLATTN_DCHECK(cond, abort_flag, status) ((cond) ? true : debug_fail((abort_flag), (status)))
+#define SOLATTN_DCHECK_STATUS(cond, status) ((cond) ? true : debug_fail_status(status))
+#else
+#define SOLATTN_DCHECK(cond, abort_flag, status) true
+#define SOLATTN_DCHECK_STATUS(cond, status) true
+#endif
 
 __device__ __forceinline__ float u2f(uint32_t x) { return __uint_as_float(x); }
 
@@ -289,12 +320,19 @@ __device__ void run_router(SmemCtl<C> &sc, const FwdParams &p, int lane) {
         uint32_t mem = 0;
 #pragma unroll
         for (int sb = 0; sb < C::NSB; ++sb) mem |= ((words[sb] >> b) & 1u) << sb;
+        if (!SOLATTN_DCHECK(w * 32 + b < nKB && pos < kMaxKeyBlocks, &sc.abort_flag, p.status)) break;
         rs.jlist[pos] = static_cast<uint16_t>(w * 32 + b);
         rs.member[pos] = static_cast<uint8_t>(mem);
         ++pos;
       }
       base += __shfl_sync(0xffffffffu, incl, 31);
     }
+#ifdef SOLATTN_DEBUG
+    if (*ab) {  // a check above failed
+      ok = false;
+      break;
+    }
+#endif
     // Statistics: kept blocks per head, and the optional keep bit-mask.
     unsigned long long kept = 0;
     for (int sb = 0; sb < C::NSB; ++sb) {
@@ -354,10 +392,14 @@ __device__ void run_producer(SmemCtl<C> &sc, const FwdParams &p, uint8_t *q_smem
       ok = false;
       return;
     }
-    mbar_arrive_expect_tx(&sc.full[slot], C::KV_BYTES);
-    uint8_t *dst = ring + slot * C::KV_BYTES;
     // a pseudo tile is BK rows of the head's pooled keys / values (zero past nKB)
     const bool pseudo = (j & kPseudoFlag) != 0;
+    if (!SOLATTN_DCHECK(pseudo ? (j & (kPseudoFlag - 1)) < p.n_pseudo : j < p.nKB, &sc.abort_flag, p.status)) {
+      ok = false;
+      return;
+    }
+    mbar_arrive_expect_tx(&sc.full[slot], C::KV_BYTES);
+    uint8_t *dst = ring + slot * C::KV_BYTES;
     const CUtensorMap *map = pseudo ? (is_v ? tm_vp : tm_kp) : (is_v ? tm_v : tm_k);
     const int row = (j & (kPseudoFlag - 1)) * C::BK;
 #pragma unroll
@@ -374,6 +416,10 @@ __device__ void run_producer(SmemCtl<C> &sc, const FwdParams &p, uint8_t *q_smem
     if (item < 0) break;
     const int bh = item / p.items_per_head;
     const int row0 = (item - bh * p.items_per_head) * C::TILE_M;
+    if (!SOLATTN_DCHECK(item < p.n_items && row0 < p.N, &sc.abort_flag, p.status)) {
+      ok = false;
+      break;
+    }
     const int qb = q_it & 1;
     if (!mbar_wait(&sc.q_empty[qb], ((q_it >> 1) & 1) ^ 1, p.timeout_ns, ab)) { ok = false; break; }
     mbar_arrive_expect_tx(&sc.q_full[qb], C::Q_TILE_BYTES);
@@ -663,6 +709,11 @@ __device__ void run_softmax(SmemCtl<C> &sc, const FwdParams &p, uint32_t tmem, i
     for (int u = w; u < n; u += 2) {
       const uint32_t mem = rs.member[u];
       const int j = rs.jlist[u];
+      if (!SOLATTN_DCHECK((j & kPseudoFlag) ? (j & (kPseudoFlag - 1)) < p.n_pseudo : j < p.nKB, &sc.abort_flag,
+                          p.status)) {
+        ok = false;
+        break;
+      }
       if (!wait(&sc.s_full[w], s_ph)) break;
       s_ph ^= 1;
       // The group that produced this S (O += P V of position u - 2, then S of position u)
@@ -676,36 +727,21 @@ __device__ void run_softmax(SmemCtl<C> &sc, const FwdParams &p, uint32_t tmem, i
       float lsum = 0.f;
       if (!TOKEN || !(j & kPseudoFlag)) {
         // One pass over the row of S held in registers: all BK columns are loaded at once
-        // (BK / 32 TMEM loads, one wait), the row maximum is a tree of three-input max
-        // instructions, and the exponentials go back to TMEM as fp16 pairs, 16 columns per
-        // store. The reference max only moves when the row maximum exceeds it by more than
-        // the slack (O and l are then rescaled once, below), so P never needs rescaling.
+        // (BK / 32 TMEM loads, one wait) and the exponentials go back to TMEM as fp16 pairs,
+        // 16 columns per store. Once every row of the warp has a reference max, the tile is
+        // first exponentiated against it without the row maximum: that is exact whatever the
+        // reference, as long as no P value overflows fp16, and a row sum <= 2^15 bounds every
+        // value by 2^15 < 65504. A warp where some row's sum is larger (or infinite) takes the
+        // row maxima (a tree of three-input max instructions) and redoes the tile, as the
+        // first tile of a row does: the reference moves when the maximum exceeds it by more
+        // than the slack (O and l are then rescaled once, below), so P never needs rescaling.
+        // A row sum above 2^15 implies a maximum more than log2(2^15 / BK) >= 8 above the
+        // reference, so such a row's reference always moves.
         constexpr int NCH = BK / 32;
         const bool rk = (mem & row_bit) != 0;  // warp-uniform (a warp's rows share a query block)
         const int ncol = (j == p.nKB - 1) ? (p.N - j * BK) : BK;
-        float mx = -CUDART_INF_F;
         uint32_t x[BK];
-        if (rk) {
-#pragma unroll
-          for (int c = 0; c < NCH; ++c) tmem_ld32(s_addr + c * 32, *reinterpret_cast<uint32_t(*)[32]>(x + c * 32));
-          tmem_wait_ld();
-          reg_fence<BK>(x);
-          if (ncol < BK) {  // ragged last key block: columns past N are not keys
-#pragma unroll
-            for (int e = 0; e < BK; ++e)
-              if (e >= ncol) x[e] = __float_as_uint(-CUDART_INF_F);
-          }
-          mx = max_tree_bits<BK>(x);
-        }
-        const float mxs = mx * sc_log2;
-        if (mxs > m_ref + kRescaleSlack) {
-          if (m_ref != -CUDART_INF_F) alpha = ex2_approx(m_ref - mxs);
-          m_ref = mxs;
-        }
-        const float neg_m = (m_ref == -CUDART_INF_F) ? 0.f : -m_ref;
-        if (rk) {
-          // Packed fp32 pairs; the pairs kPolyMask selects go through the FMA-pipe exp2. Masked
-          // columns hold -inf and give 0 (MUFU) or 2^-125 (polynomial), i.e. 0 in fp16.
+        auto exp_all = [&](float neg_m) {
           const uint64_t scp = f2(sc_log2, sc_log2);
           const uint64_t nmp = f2(neg_m, neg_m);
           uint64_t acc[4] = {f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f)};
@@ -734,14 +770,44 @@ __device__ void run_softmax(SmemCtl<C> &sc, const FwdParams &p, uint32_t tmem, i
           f2_split(acc[1], s2, s3);
           f2_split(acc[2], s4, s5);
           f2_split(acc[3], s6, s7);
-          lsum = ((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7));
-        } else {
-          // This row's query block does not keep the block (two query blocks per tile): P = 0.
-          uint32_t pk[16];
+          return ((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7));
+        };
+        bool done = false;
+        float mx = -CUDART_INF_F;
+        if (rk) {
 #pragma unroll
-          for (int e = 0; e < 16; ++e) pk[e] = 0u;
+          for (int c = 0; c < NCH; ++c) tmem_ld32(s_addr + c * 32, *reinterpret_cast<uint32_t(*)[32]>(x + c * 32));
+          tmem_wait_ld();
+          reg_fence<BK>(x);
+          if (ncol < BK) {  // ragged last key block: columns past N are not keys
 #pragma unroll
-          for (int c = 0; c < NCH; ++c) tmem_st16(s_addr + c * 16, pk);
+            for (int e = 0; e < BK; ++e)
+              if (e >= ncol) x[e] = __float_as_uint(-CUDART_INF_F);
+          }
+          if (__all_sync(0xffffffffu, m_ref != -CUDART_INF_F)) {
+            lsum = exp_all(-m_ref);
+            done = __all_sync(0xffffffffu, lsum <= kSpecRowSumLimit);
+            if (!done) tmem_wait_st();
+          }
+          if (!done) mx = max_tree_bits<BK>(x);
+        }
+        if (!done) {
+          const float mxs = mx * sc_log2;
+          if (mxs > m_ref + kRescaleSlack) {
+            if (m_ref != -CUDART_INF_F) alpha = ex2_approx(m_ref - mxs);
+            m_ref = mxs;
+          }
+          const float neg_m = (m_ref == -CUDART_INF_F) ? 0.f : -m_ref;
+          if (rk) {
+            lsum = exp_all(neg_m);
+          } else {
+            // This row's query block does not keep the block (two query blocks per tile): P = 0.
+            uint32_t pk[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) pk[e] = 0u;
+#pragma unroll
+            for (int c = 0; c < NCH; ++c) tmem_st16(s_addr + c * 16, pk);
+          }
         }
       } else if constexpr (TOKEN) {
         softmax_pseudo_tile<BK>(s_addr, j & (kPseudoFlag - 1), rs.kmask[sb], p.N, p.nKB, sc_log2, m_ref, alpha, lsum);

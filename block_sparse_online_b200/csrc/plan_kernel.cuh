@@ -195,7 +195,10 @@ __global__ void __launch_bounds__(256, 2) plan_kernel(const FwdParams p, uint32_
     if (gauss && kept == 0 && lane == 0) atomicOr(&mrow[top_j >> 5], 1u << (top_j & 31));
     __syncwarp();
     uint32_t *kw = keep_out + (static_cast<size_t>(bh) * nQB + qb) * nW;
-    for (int w = lane; w < nW; w += 32) kw[w] = mrow[w];
+    // bits past nKB stay clear: the router turns every set bit into a key block index
+    for (int w = lane; w < nW; w += 32)
+      if (SOLATTN_DCHECK_STATUS(w < nW - 1 || (nKB & 31) == 0 || (mrow[w] >> (nKB & 31)) == 0u, p.status))
+        kw[w] = mrow[w];
     if (correct) {
       float l = 0.f;
       for (int j = lane; j < nKB; j += 32) {
@@ -275,7 +278,8 @@ __global__ void __launch_bounds__(256, 2) plan_kernel(const FwdParams p, uint32_
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, off);
-    if (lane == 0) cost[bh * p.items_per_head + qb0 / SUBQ + it] = cnt;
+    const int item = bh * p.items_per_head + qb0 / SUBQ + it;
+    if (lane == 0 && SOLATTN_DCHECK_STATUS(item < p.n_items && cnt <= nKB, p.status)) cost[item] = cnt;
   }
   // The last CTA to finish orders the items: groups of `group_heads` consecutive heads in
   // head order (the group's K/V stays resident in L2), and within a group the costliest
@@ -332,7 +336,7 @@ __global__ void __launch_bounds__(256, 2) plan_kernel(const FwdParams p, uint32_
     __syncthreads();
     for (int i = threadIdx.x; i < i1 - i0; i += blockDim.x) {
       const int pos = atomicAdd(&hist[cs[i]], 1);
-      order[i0 + pos] = i0 + i;
+      if (SOLATTN_DCHECK_STATUS(pos < i1 - i0, p.status)) order[i0 + pos] = i0 + i;
     }
     __syncthreads();
   }

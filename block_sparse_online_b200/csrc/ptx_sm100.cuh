@@ -355,7 +355,9 @@ __device__ __forceinline__ void exp2_poly_x2(float x0, float x1, float &y0, floa
   constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
   constexpr float c0 = 0.9999280571937561f, c1 = 0.6932609677314758f;
   constexpr float c2 = 0.2426111251115799f, c3 = 0.0551716685295105f;
-  const uint64_t x = f2(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+  // Clamped to [-125, 64]: the exponent add below stays inside fp32's exponent range, so a
+  // large input gives a large finite value (2^64) rather than a wrapped exponent.
+  const uint64_t x = f2(fminf(fmaxf(x0, -125.f), 64.f), fminf(fmaxf(x1, -125.f), 64.f));
   const uint64_t t = add2(x, f2(kShift, kShift));
   const uint64_t nf = add2(t, f2(-kShift, -kShift));
   const uint64_t fr = fma2(nf, f2(-1.f, -1.f), x);

@@ -8,6 +8,8 @@
 #include <cstring>
 #include <mutex>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "attn_kernel.cuh"
 #include "plan_kernel.cuh"
 #include "pool_kernel.cuh"
@@ -27,6 +29,15 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 int nblocks(int N, int blk) { return (N + blk - 1) / blk; }
 
 bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// NVTX range around the host code that enqueues one stage ("solattn pool", "solattn route",
+// "solattn attention", ...), for timeline tools; without a tool attached it costs a few ns.
+struct NvtxRange {
+  explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange &) = delete;
+  NvtxRange &operator=(const NvtxRange &) = delete;
+};
 
 struct WsLayout {
   size_t qbar, kbar, vbar, v16, cost, order, kmom, theta, kbar16, vbar16, corr, keep, total;
@@ -360,6 +371,7 @@ int forward_impl(const void *q, const void *k, const void *v, void *out, int B, 
       a.job[2] = PoolJob{static_cast<const __nv_bfloat16 *>(k), kbar, nullptr, Bk, nKB};
       a.njobs = 3;
     }
+    NvtxRange r("solattn pool");
     const int rcp = launch_pool(a, BH, d, nQB > nKB ? nQB : nKB, st);
     if (rcp != SOLATTN_OK) return rcp;
   }
@@ -416,6 +428,7 @@ int forward_impl(const void *q, const void *k, const void *v, void *out, int B, 
       group_heads = kPlanOrderCap / per_head > 1 ? kPlanOrderCap / per_head : 1;
     int *cost = reinterpret_cast<int *>(ws + wl.cost);
     int *order = reinterpret_cast<int *>(ws + wl.order);
+    NvtxRange r("solattn route");
     const int rp = dispatch_plan(d, Bq, Bk, p, BH, p.keep_bits, cost, order, reinterpret_cast<unsigned int *>(ws + 8),
                                  group_heads, st);
     if (rp != SOLATTN_OK) return rp;
@@ -423,8 +436,11 @@ int forward_impl(const void *q, const void *k, const void *v, void *out, int B, 
   }
   if (ev_attn_begin && cudaEventRecord(static_cast<cudaEvent_t>(ev_attn_begin), st) != cudaSuccess)
     return SOLATTN_ECUDA;
-  const int rl = dispatch(d, Bq, Bk, mq, mk, mv, mkp, mvp, p, di.sms, st);
-  if (rl != SOLATTN_OK) return rl;
+  {
+    NvtxRange r("solattn attention");
+    const int rl = dispatch(d, Bq, Bk, mq, mk, mv, mkp, mvp, p, di.sms, st);
+    if (rl != SOLATTN_OK) return rl;
+  }
   if (ev_attn_end && cudaEventRecord(static_cast<cudaEvent_t>(ev_attn_end), st) != cudaSuccess)
     return SOLATTN_ECUDA;
   return SOLATTN_OK;
@@ -742,6 +758,7 @@ const char *solattn_strerror(int status) {
     case SOLATTN_ECUDA: return "CUDA error";
     case SOLATTN_ETIMEOUT: return "device-side wait timed out";
     case SOLATTN_EWORKSPACE: return "workspace missing, misaligned or too small";
+    case SOLATTN_EBOUNDS: return "device-side bounds check failed (debug build)";
     default: return "unknown status";
   }
 }

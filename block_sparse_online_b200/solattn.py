@@ -12,6 +12,9 @@ import os
 import torch
 
 _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsolattn.so")
+# The build with the kernels' device-side bounds checks (python -m block_sparse_online_b200.build
+# --debug): same exports, failed checks reported as SOLATTN_EBOUNDS.
+DEBUG_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsolattn_debug.so")
 
 SOLATTN_DENSE = 0
 SOLATTN_KEEP_DROP = 1
@@ -24,6 +27,7 @@ SOLATTN_EUNSUPPORTED = -2
 SOLATTN_ECUDA = -3
 SOLATTN_ETIMEOUT = -4
 SOLATTN_EWORKSPACE = -5
+SOLATTN_EBOUNDS = -6
 MAX_KEY_BLOCKS = 1024
 
 EXPORTS = ("solattn_workspace_size", "solattn_pool", "solattn_forward", "solattn_forward_events",
@@ -52,11 +56,11 @@ class _Route(ctypes.Structure):  # solattn_route
                 ("correction", ctypes.c_int)]
 
 
-def _load():
-    if not os.path.exists(_LIB_PATH):
-        raise ImportError(f"libsolattn.so is not built ({_LIB_PATH}); run "
-                          "`python -m block_sparse_online_b200.build`")
-    lib = ctypes.CDLL(_LIB_PATH)
+def _load(path=_LIB_PATH):
+    if not os.path.exists(path):
+        raise ImportError(f"{os.path.basename(path)} is not built ({path}); run "
+                          "`python -m block_sparse_online_b200.build`" + (" --debug" if path == DEBUG_LIB_PATH else ""))
+    lib = ctypes.CDLL(path)
     i, sz, vp, f = ctypes.c_int, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_float
     lib.solattn_workspace_size.argtypes = [i, i, i, i, i, i]
     lib.solattn_workspace_size.restype = sz
@@ -98,10 +102,21 @@ def _load():
 
 
 _lib = _load()
+_lib_path = _LIB_PATH
 
 
 def library_path() -> str:
-    return _LIB_PATH
+    return _lib_path
+
+
+def load_library(path: str = _LIB_PATH) -> str:
+    """Route every call of this module through the library at `path` (the release build by
+    default, or DEBUG_LIB_PATH); returns the path that was active before."""
+    global _lib, _lib_path
+    lib = _load(path)
+    prev = _lib_path
+    _lib, _lib_path = lib, path
+    return prev
 
 
 def strerror(status: int) -> str:

@@ -69,7 +69,9 @@ typedef enum {
   SOLATTN_EUNSUPPORTED = -2, /* d or Bq/Bk not in {64,128}, nKB > 1024, B*H > 65535, no sm_100 device */
   SOLATTN_ECUDA = -3,        /* a CUDA runtime or driver call failed                          */
   SOLATTN_ETIMEOUT = -4,     /* a device-side wait ran past its limit (reported by get_status) */
-  SOLATTN_EWORKSPACE = -5    /* workspace pointer null/misaligned or smaller than required     */
+  SOLATTN_EWORKSPACE = -5,   /* workspace pointer null/misaligned or smaller than required     */
+  SOLATTN_EBOUNDS = -6       /* a device-side bounds check failed (libsolattn_debug.so only:
+                                the build with -DSOLATTN_DEBUG; reported by get_status)        */
 } solattn_status;
 
 /* Per-call statistics (device pointers). */

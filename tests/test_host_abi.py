@@ -34,9 +34,27 @@ def test_library_exports_every_declared_symbol():
     assert set(declared_functions()) == set(solattn.EXPORTS)
 
 
+def test_debug_library_exports_every_declared_symbol():
+    """The bounds-checked build (-DSOLATTN_DEBUG) is the same boundary: it is built here if
+    it is missing (nvcc cross-compiles without a GPU) and loaded without one."""
+    if not os.path.exists(solattn.DEBUG_LIB_PATH):
+        from block_sparse_online_b200 import build
+        try:
+            build.nvcc()
+        except RuntimeError:
+            pytest.skip("nvcc not available to build the debug library")
+        build.build(debug=True)
+    lib = ctypes.CDLL(solattn.DEBUG_LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    assert lib.solattn_workspace_size(1, 12, 32760, 128, 128, 128) == \
+        solattn.solattn_workspace_size(1, 12, 32760, 128, 128, 128)
+
+
 def test_strerror():
     assert solattn.strerror(0) == "ok"
     assert "timed out" in solattn.strerror(solattn.SOLATTN_ETIMEOUT)
+    assert "bounds check" in solattn.strerror(solattn.SOLATTN_EBOUNDS)
     assert solattn.strerror(12345) == "unknown status"
 
 
