@@ -31,7 +31,7 @@
 
 namespace solattn {
 
-constexpr int kPlanQG = 16;       // query blocks per CTA
+constexpr int kPlanQG = 12;       // query blocks per CTA
 constexpr int kPlanWarps = 8;     // 256 threads
 constexpr int kPlanBatch = 4;     // pooled-key float4 loads per batch (step 1; two batches in flight)
 constexpr int kPlanOrderCap = 4096;  // most work items in one ordering group (host-enforced)
@@ -294,7 +294,7 @@ __global__ void __launch_bounds__(256, 2) plan_kernel(const FwdParams p, uint32_
   const int nbins = nKB + 1;  // cost in [0, nKB]
   // The group's costs are copied to shared memory first (one round of independent loads
   // instead of a dependent global load per pass), into the dynamic shared memory this CTA
-  // no longer needs: at least plan_smem_bytes<64>(1) / 4 = 9792 ints, while the host keeps
+  // no longer needs: at least plan_smem_bytes<64>(1) / 4 = 7344 ints, while the host keeps
   // a group to max(items_per_head, kPlanOrderCap) <= 4096 items.
   int *cs = reinterpret_cast<int *>(plan_smem);
   for (int h0 = 0; h0 < BH; h0 += group_heads) {
